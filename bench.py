@@ -1,0 +1,456 @@
+#!/usr/bin/env python
+"""Benchmark of paged quantised-KV attention on B200 (one JSON line on rank 0).
+
+A step is one call of the whole hot path (fused attention kernel, plus the
+log-sum-exp combine kernel when the planner splits the KV) over one batch of
+seeded synthetic input whose cache is already resident in HBM.  Between steps
+the L2 cache (126 MB) is flushed by writing a 256 MB buffer, outside the timed
+spans; each step is timed with CUDA events on the launching stream.
+
+Headline workload (N=1): INT4 packed decode, B=16, q_len=1, 32 query / 8 KV
+heads, head_size 128, block_size 16, seqlens_k ~ U[512, 4096].  The other
+workloads are reported under "workloads" with the same method.
+
+Metric: effective HBM bandwidth = algorithmic bytes per call / time per call
+(KV bytes of the sequences with new tokens + Q in + out + scales + block-table
+entries read + lengths), plus us/call and tokens/s.
+
+--impl reference times the FP64 CPU oracle (single thread) on a bounded sample
+of the same workload, which is the comparison arm of this build.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+HEADLINE = "c2_int4_decode"
+EXTRA = ["c3_int8_long_split", "c5_fp8_large_batch", "c4_ragged_prefill_int8", "c1_tiny_int8"]
+L2_FLUSH_BYTES = 256 << 20
+
+
+def algorithmic_bytes(w: dict) -> dict:
+    """Bytes the method must move per call (the measurement section's formula)."""
+    D, H, Hk, bs = w["head_size"], w["num_heads"], w["kv_num_heads"], w["block_size"]
+    chs = workloads.cache_bytes_per_row(w["kv_dtype"], D)
+    ql = np.diff(w["cu_seqlens_q"]).astype(np.int64)
+    L = w["seqlens_k"].astype(np.int64)
+    act = ql > 0
+    kv = int((L[act] * Hk * 2 * chs).sum())
+    T = int(w["cu_seqlens_q"][-1])
+    qo = T * H * D * (2 + 2)
+    scales = 2 * Hk * D * 4
+    bt = int(((L[act] + bs - 1) // bs).sum()) * 4
+    meta = 4 * w["batch"] + 4 * (w["batch"] + 1)
+    total = kv + qo + scales + bt + meta
+    return dict(total=total, kv=kv, qo=qo, tokens=T, fwd=total)
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("pa_attention.cu", "pa_device.cuh"):
+        with open(os.path.join(ROOT, "paged_quantized_kv_attention_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(name: str):
+    """DRAM bytes per launch from the committed ncu summary, if it still matches
+    the kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(name)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("kernel_source_sha") != kernel_source_sha():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except (OSError, ValueError, KeyError):
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML while the timed region runs."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # NVML missing: report nulls
+            self.max_mhz = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.reasons |= int(r) & ~0x1
+            except Exception:
+                pass
+            time.sleep(0.001)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+def setup(w: dict, dev: str):
+    import paged_quantized_kv_attention_b200 as pa
+    from_np = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)  # noqa: E731
+    d = dict(q=w["q"].to(dev), k_cache=from_np(w["k_cache"]), v_cache=from_np(w["v_cache"]),
+             k_scale=from_np(w["k_scale"].astype(np.float32)),
+             v_scale=from_np(w["v_scale"].astype(np.float32)),
+             block_table=from_np(w["block_table"]), seqlens_k=from_np(w["seqlens_k"]),
+             cu_seqlens_q=from_np(w["cu_seqlens_q"]))
+    p = pa.make_params(batch=w["batch"], num_heads=w["num_heads"], kv_num_heads=w["kv_num_heads"],
+                       head_size=w["head_size"], block_size=w["block_size"],
+                       num_blocks=w["num_blocks"], max_blocks_per_seq=w["max_blocks_per_seq"],
+                       kv_dtype=w["kv_dtype"], q_dtype=w["q_dtype"], out_dtype=w["out_dtype"],
+                       causal=w["causal"])
+    ws_bytes = pa.paged_attn_plan(w["cu_seqlens_q"], w["seqlens_k"], p)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    pa.paged_attn_workspace_init(ws, ws_bytes)
+    p.workspace = ws.data_ptr()
+    odt = torch.bfloat16 if w["out_dtype"] == 1 else torch.float16
+    T = int(w["cu_seqlens_q"][-1])
+    d["out"] = torch.empty((T, w["num_heads"], w["head_size"]), dtype=odt, device=dev)
+    d["ws"] = ws
+    return d, p
+
+
+def _event_handles(evs):
+    import ctypes
+    arr = (ctypes.c_void_p * 2)(evs[0].cuda_event, evs[1].cuda_event)
+    return arr
+
+
+def time_device(w, d, p, steps, warmup, flush):
+    """Per-step device time of the whole call and of the fused kernel (ms lists)."""
+    import ctypes
+
+    import paged_quantized_kv_attention_b200 as pa
+    stream = torch.cuda.current_stream()
+    args = (d["q"], d["k_cache"], d["v_cache"], d["k_scale"], d["v_scale"], d["block_table"],
+            d["seqlens_k"], d["cu_seqlens_q"], d["out"])
+    for _ in range(warmup):
+        flush.zero_()
+        pa.paged_attn_forward(*args, p, stream)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for e in ev:  # create the events before handing their handles to the library
+        for x in e:
+            x.record(stream)
+    torch.cuda.synchronize()
+    holders = []
+    for i in range(steps):
+        flush.zero_()  # L2 flush, between the timed spans
+        h = _event_handles(ev[i][:2])
+        holders.append(h)
+        p.profile_events = ctypes.cast(h, ctypes.c_void_p)
+        pa.paged_attn_forward(*args, p, stream)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    p.profile_events = None
+    call_ms = [ev[i][0].elapsed_time(ev[i][2]) for i in range(steps)]
+    kern_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(steps)]
+    return call_ms, kern_ms
+
+
+def time_e2e(w, d, p, steps, warmup, flush):
+    """Through the public API with host buffers: H2D of the step's inputs from pinned
+    memory, host planning, forward, D2H of the output; device-timed per step."""
+    import paged_quantized_kv_attention_b200 as pa
+    stream = torch.cuda.current_stream()
+    host = {k: d[k].cpu().pin_memory() for k in ("q", "block_table", "seqlens_k", "cu_seqlens_q")}
+    cu_h, sk_h = w["cu_seqlens_q"].copy(), w["seqlens_k"].copy()
+    out_h = torch.empty(d["out"].shape, dtype=d["out"].dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+
+    def one():
+        for k, t in host.items():
+            d[k].copy_(t, non_blocking=True)
+        pa.paged_attn_plan(cu_h, sk_h, p)
+        pa.paged_attn_forward(d["q"], d["k_cache"], d["v_cache"], d["k_scale"], d["v_scale"],
+                              d["block_table"], d["seqlens_k"], d["cu_seqlens_q"], d["out"], p,
+                              stream)
+        out_h.copy_(d["out"], non_blocking=True)
+
+    for _ in range(warmup):
+        flush.zero_()
+        one()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        one()
+        e1.record(stream)
+        e1.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    return ms, h2d, d2h
+
+
+def cpu_oracle_sample(w: dict, budget_s: float):
+    """The FP64 oracle as it stands, single-threaded, over whole sequences of the
+    workload until about budget_s seconds of CPU work; returns (GB/s, detail)."""
+    import oracle
+    ov = workloads.oracle_view(w)
+    cu = w["cu_seqlens_q"]
+    done_bytes, t_used, seqs, keys = 0, 0.0, 0, 0
+    for b in range(w["batch"]):
+        if cu[b + 1] == cu[b]:
+            continue
+        s = sub_problem(ov, b)
+        t0 = time.perf_counter()
+        oracle.paged_attn(s)
+        t_used += time.perf_counter() - t0
+        done_bytes += algorithmic_bytes(s)["total"]
+        seqs += 1
+        keys += int(s["seqlens_k"][0])
+        if t_used >= budget_s:
+            break
+    gbs = done_bytes / t_used / 1e9 if t_used > 0 else None
+    return gbs, dict(seconds=round(t_used, 3), sequences=seqs, keys=keys, bytes=done_bytes)
+
+
+def sub_problem(w: dict, b: int) -> dict:
+    cu = w["cu_seqlens_q"]
+    s = dict(w)
+    s["batch"] = 1
+    s["block_table"] = np.ascontiguousarray(w["block_table"][b:b + 1])
+    s["seqlens_k"] = np.ascontiguousarray(w["seqlens_k"][b:b + 1])
+    s["cu_seqlens_q"] = np.array([0, cu[b + 1] - cu[b]], dtype=np.int32)
+    s["q"] = w["q"][int(cu[b]):int(cu[b + 1])]
+    return s
+
+
+def measure(name: str, steps: int, warmup: int, dev: str, flush, with_e2e: bool):
+    w = workloads.make(name)
+    ab = algorithmic_bytes(w)
+    d, p = setup(w, dev)
+    call_ms, kern_ms = time_device(w, d, p, steps, warmup, flush)
+    call = statistics.mean(call_ms)
+    kern = statistics.mean(kern_ms)
+    peak, peak_kind = measured_peaks()
+    res = dict(w=w, ab=ab, p=p, call_ms=call, kern_ms=kern,
+               value=ab["total"] / (call * 1e-3) / 1e9,
+               kernel_gbs=ab["fwd"] / (kern * 1e-3) / 1e9, peak=peak, peak_kind=peak_kind,
+               launches_per_step=1 + (1 if p.num_splits > 1 else 0))
+    if with_e2e:
+        e2e_ms, h2d, d2h = time_e2e(w, d, p, max(5, steps // 2), 2, flush)
+        res["e2e"] = dict(value=ab["total"] / (statistics.mean(e2e_ms) * 1e-3) / 1e9,
+                          unit="GB/s", h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
+                          ms_per_step=statistics.mean(e2e_ms))
+    del d
+    torch.cuda.empty_cache()
+    return res
+
+
+def summary_of(name, r):
+    return {"workload": name, "desc": workloads.DESCRIPTIONS[name],
+            "gbs": round(r["value"], 1), "us_per_call": round(r["call_ms"] * 1e3, 2),
+            "tokens_per_s": round(r["ab"]["tokens"] / (r["call_ms"] * 1e-3), 1),
+            "kernel_us": round(r["kern_ms"] * 1e3, 2),
+            "kernel_gbs": round(r["kernel_gbs"], 1),
+            "kernel_frac_of_%s_peak" % r["peak_kind"]: round(r["kernel_gbs"] / r["peak"], 3),
+            "num_splits": r["p"].num_splits, "algorithmic_bytes": r["ab"]["total"]}
+
+
+def run_ours(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    dev = "cuda:%d" % torch.cuda.current_device()
+    import paged_quantized_kv_attention_b200 as pa
+    pa.lib()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    # headline workload: identical per-rank replica (weak scaling, no collective on the path)
+    w_name = args.workload
+    sampler = ClockSampler(torch.cuda.current_device())
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        r = measure(w_name, args.steps, args.warmup, dev, flush, with_e2e=True)
+    torch.cuda.synchronize()
+    if dist is not None:
+        t = torch.tensor([r["call_ms"], r["e2e"]["ms_per_step"]], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.barrier()
+        r["call_ms"], r["e2e"]["ms_per_step"] = float(t[0]), float(t[1])
+    extra = {}
+    if not args.no_extra:
+        for name in EXTRA:
+            if name == w_name:
+                continue
+            rr = measure(name, max(3, min(args.steps, 20)), args.warmup, dev, flush,
+                         with_e2e=False)
+            extra[name] = summary_of(name, rr)
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+    ab = r["ab"]
+    value = world * ab["total"] / (r["call_ms"] * 1e-3) / 1e9
+    e2e_value = world * ab["total"] / (r["e2e"]["ms_per_step"] * 1e-3) / 1e9
+    cpu = None
+    if world == 1 and not args.no_cpu:
+        gbs, det = cpu_oracle_sample(r["w"], args.cpu_seconds)
+        cpu = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": "FP64 oracle, one thread, whole sequences of the same workload in order "
+                         "until ~%.0f s: %d sequences, %d keys, %.1f s" %
+                         (args.cpu_seconds, det["sequences"], det["keys"], det["seconds"])}
+    line = {
+        "metric": "paged quantized-KV attention: effective HBM GB/s (% of ~8 TB/s), us/call",
+        "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(r["call_ms"], 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic (seeded numpy PCG64; cache resident in HBM)",
+        "config": {"workload": w_name, "desc": workloads.DESCRIPTIONS[w_name],
+                   "kv_dtype": workloads.KV_NAMES[r["w"]["kv_dtype"]],
+                   "global_batch": r["w"]["batch"] * world, "seq_len": int(r["w"]["seqlens_k"].max()),
+                   "parallelism": "replicas x%d" % world,
+                   "l2": "flushed between steps (256 MB write), per-step CUDA events",
+                   "num_splits": r["p"].num_splits, "blocks_per_split": r["p"].blocks_per_split},
+        "us_per_call": round(r["call_ms"] * 1e3, 3),
+        "tokens_per_s": round(world * ab["tokens"] / (r["call_ms"] * 1e-3), 1),
+        "pct_of_8tbs": round(100 * value / world / 8000.0, 2),
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": r["e2e"]["h2d_bytes_per_step"],
+                "d2h_bytes_per_step": r["e2e"]["d2h_bytes_per_step"],
+                "us_per_step": round(r["e2e"]["ms_per_step"] * 1e3, 2)},
+        "gpu_launches": args.steps * r["launches_per_step"],
+        "roofline": {"bound": "hbm", "achieved": round(r["kernel_gbs"], 1),
+                     "peak": r["peak"], "unit": "GB/s",
+                     "frac": round(r["kernel_gbs"] / r["peak"], 4),
+                     "peak_kind": r["peak_kind"],
+                     "kernel": "pa_fwd_kernel", "kernel_us": round(r["kern_ms"] * 1e3, 3),
+                     "algorithmic_bytes_per_launch": ab["fwd"],
+                     "traffic": ncu_traffic(w_name)},
+        "clocks": sampler.summary(),
+        "cpu_baseline": cpu,
+        "workloads": extra,
+    }
+    print(json.dumps(line))
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The comparison arm: the FP64 oracle on the host cores, rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    w = workloads.make(args.workload)
+    ov = workloads.oracle_view(w)
+    cu = w["cu_seqlens_q"]
+    seqs = [b for b in range(w["batch"]) if cu[b + 1] > cu[b]]
+    for i in range(args.warmup):
+        oracle.paged_attn(sub_problem(ov, seqs[i % len(seqs)]))
+    t_total, bytes_total, keys = 0.0, 0, 0
+    for i in range(args.steps):
+        s = sub_problem(ov, seqs[i % len(seqs)])
+        t0 = time.perf_counter()
+        oracle.paged_attn(s)
+        t_total += time.perf_counter() - t0
+        bytes_total += algorithmic_bytes(s)["total"]
+        keys += int(s["seqlens_k"][0])
+    value = bytes_total / t_total / 1e9
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    sample = ("FP64 oracle, one thread, one whole sequence of %s per step (%d steps, %d keys)"
+              % (args.workload, args.steps, keys))
+    line = {"impl": "reference",
+            "metric": "paged quantized-KV attention: effective HBM GB/s (% of ~8 TB/s), us/call",
+            "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * t_total / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded numpy PCG64)",
+            "config": {"workload": args.workload, "desc": workloads.DESCRIPTIONS[args.workload]},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=HEADLINE, choices=workloads.NAMES)
+    ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,199 @@
+/*
+ * paged_attn.h -- C ABI of the B200 (sm_100a) paged quantised-KV attention library
+ * (libpagedattn.so).
+ *
+ * Operation.  Grouped-query attention of the new tokens of a ragged batch over a
+ * paged low-precision KV cache:
+ *
+ *     out = softmax(scale * Q * dequant(K)^T + causal mask) * dequant(V)
+ *
+ * Sources (blog summaries of merged pull requests; cited by title and section):
+ *  - "ONNX Runtime: INT4 Paged KV Cache ... memory optimisation" (onnxruntime
+ *    PR 32515), Code analysis 2: cache shape (num_blocks, block_size,
+ *    kv_num_heads, cache_head_size) with cache_head_size = (head_size + 1) / 2 for
+ *    packed INT4 and head_size otherwise; Code analysis 3: the per-channel K
+ *    scale is folded into Q, normalised by the power of two of max|k_scale| so
+ *    fp16 cannot overflow.
+ *  - "ONNX Runtime: Tensor-Core DynamicSparseAttention for INT8-KV cache"
+ *    (onnxruntime PR 33707), Code analysis 1: INT8 kept raw until it is
+ *    converted to FP16 in registers right before the tensor-core MMA, FP32
+ *    accumulation.
+ *  - "[ONNX Runtime] PagedAttention FA path: exact max_query_len" (onnxruntime
+ *    PR 28409), Code analysis 1-2: the launch is sized by the exact host-side
+ *    max over b of cu_seqlens_q[b+1] - cu_seqlens_q[b]; sequences with zero new
+ *    tokens are legal.
+ *  - "Escaping the SGEMM trap: GQA GEMV decode kernel" (onnxruntime PR 29216),
+ *    Code analysis 2: flash decoding splits one sequence's keys across workers
+ *    when batch x heads underfills the machine, with a partials buffer.
+ *  - "FlashInfer FP8 KV-Cache Prefill ... Repacking" (flashinfer PR 3485):
+ *    1-byte FP8 KV cache (read here as OCP e4m3fn).
+ *
+ * Readings where the pages are silent (all of them are properties of this ABI):
+ *  - seqlens_k[b] counts every key of sequence b, the new tokens included; the
+ *    past length is seqlens_k[b] - q_b (q_b = new tokens of b).
+ *  - Causal mask is bottom-right aligned: new token i of b sees keys
+ *    t <= seqlens_k[b] - q_b + i.  For decode (q_b = 1) that is every key.
+ *  - Query head h uses KV head h / (num_heads / kv_num_heads).
+ *  - INT4: channel 2j is the low nibble of byte j, channel 2j+1 the high nibble,
+ *    4-bit two's complement in [-8, 7].
+ *  - Dequantisation is symmetric: value = scale[kv, d] * code, scales fp32
+ *    [kv_num_heads, head_size], shared by every token and block.
+ *
+ * Memory layouts (all row-major, all device memory unless the name says _host):
+ *  q, out        [total_q, num_heads, head_size] fp16 or bf16, tokens packed by
+ *                cu_seqlens_q (sequence b owns rows cu[b] .. cu[b+1]-1).
+ *  k_cache,
+ *  v_cache       [num_blocks, block_size, kv_num_heads, cache_head_size] bytes.
+ *                Base address 16-byte aligned.
+ *  k_scale,
+ *  v_scale       [kv_num_heads, head_size] fp32.
+ *  block_table   [batch, max_blocks_per_seq] int32; entry (b, l) is the physical
+ *                block holding keys l*block_size .. l*block_size+block_size-1.
+ *  seqlens_k     [batch] int32.
+ *  cu_seqlens_q  [batch + 1] int32, cu[0] = 0, non-decreasing.
+ *
+ * Ownership and state.  The caller owns every buffer, the workspace included.
+ * The library allocates no memory and keeps no state between calls; every call
+ * is asynchronous on the given stream (a cudaStream_t passed as void*; NULL is
+ * the legacy default stream).  No exception crosses the ABI: each entry point
+ * returns a pa_status, and paged_attn_last_error() gives a message for the last
+ * failing call on the calling thread.
+ *
+ * Errors.  Argument and contract violations are detected on the host before
+ * any launch and return PA_ERR_INVALID_ARG / PA_ERR_UNSUPPORTED /
+ * PA_ERR_WORKSPACE.  A launch failure returns PA_ERR_CUDA.  Conditions that
+ * only the device can see (a block-table entry outside [0, num_blocks), a
+ * non-finite k_scale, device lengths that contradict the plan, a pipeline wait
+ * that timed out) never fault the GPU: the kernel reads zeros instead, finishes,
+ * and ORs a bit into the sticky error word at the start of the workspace, which
+ * paged_attn_read_device_error() returns.
+ */
+#ifndef PAGED_ATTN_H
+#define PAGED_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = -1,     /* bad pointer, size, or contract violation */
+  PA_ERR_UNSUPPORTED = -2,     /* valid request outside the compiled set */
+  PA_ERR_WORKSPACE = -3,       /* workspace missing or smaller than planned */
+  PA_ERR_BAD_BLOCK_TABLE = -4, /* device error word: block id out of range */
+  PA_ERR_CUDA = -5,            /* CUDA runtime / launch error */
+  PA_ERR_DEVICE = -6           /* device error word: other device-side condition */
+} pa_status;
+
+typedef enum { PA_KV_INT8 = 0, PA_KV_INT4 = 1, PA_KV_FP8_E4M3 = 2 } pa_kv_dtype;
+typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
+
+/* Bits of the device error word (see paged_attn_read_device_error). */
+#define PA_DEVERR_BAD_BLOCK 0x1u   /* block_table entry outside [0, num_blocks) */
+#define PA_DEVERR_TIMEOUT 0x2u     /* an mbarrier wait exceeded its time bound */
+#define PA_DEVERR_BAD_SCALE 0x4u   /* max |k_scale| of a KV head is not finite */
+#define PA_DEVERR_BAD_LENGTH 0x8u  /* device seqlens/cu_seqlens contradict the plan */
+
+typedef struct {
+  /* ---- problem description: filled by the caller ---- */
+  int batch;              /* B >= 0 */
+  int num_heads;          /* H, query heads */
+  int kv_num_heads;       /* Hk, H % Hk == 0 */
+  int head_size;          /* D: 64 or 128 */
+  int block_size;         /* tokens per cache block: 16 or 32 */
+  int num_blocks;         /* physical blocks in each cache pool */
+  int max_blocks_per_seq; /* columns of block_table */
+  int kv_dtype;           /* pa_kv_dtype */
+  int q_dtype;            /* pa_dtype of q */
+  int out_dtype;          /* pa_dtype of out */
+  float softmax_scale;    /* 0 -> 1/sqrt(head_size) */
+  int causal;             /* 1: bottom-right causal mask for new tokens; 0: none */
+  int num_sms;            /* 0 -> SM count of the current device (148 if none) */
+  int split_blocks;       /* 0: planner decides; > 0: force this many KV blocks per
+                             split; < 0: never split */
+  /* ---- filled by paged_attn_plan ---- */
+  int total_q;            /* cu_seqlens_q[batch] */
+  int max_query_len;      /* exact max_b (cu[b+1] - cu[b]) */
+  int max_seqlen_k;       /* max_b seqlens_k[b] */
+  int rows_per_cta;       /* query rows (tokens x group heads) per CTA: 8 or 16 */
+  int num_row_groups;     /* ceil(max_query_len * H/Hk / rows_per_cta) */
+  int num_splits;         /* KV splits of the longest sequence (1 = no split) */
+  int blocks_per_split;   /* KV blocks per split */
+  size_t workspace_bytes; /* bytes the forward call needs (>= 256) */
+  /* ---- supplied by the caller before paged_attn_forward ---- */
+  void* workspace;        /* device memory, 256-byte aligned, >= workspace_bytes,
+                             zeroed once with paged_attn_workspace_init */
+  void* profile_events;   /* optional profiling hook: NULL, or a pointer to two
+                             cudaEvent_t that paged_attn_forward records on the
+                             stream right before and right after the fused
+                             attention kernel (the combine kernel falls outside) */
+} paged_attn_params;
+
+/* Host-side planner.  Validates the problem, computes the exact max_query_len
+ * and max_seqlen_k from HOST copies of cu_seqlens_q [batch+1] and seqlens_k
+ * [batch] (the exact-max_query_len page, Code analysis 1), chooses the KV split
+ * (split-KV when B*Hk*row groups underfills the SMs and there is more than one
+ * block per sequence, after the GQA GEMV decode page's flash-decoding rule), and
+ * reports the workspace size.  Launches nothing; needs no GPU.  Contract checks:
+ * cu[0] == 0, 0 <= q_b <= seqlens_k[b] <= max_blocks_per_seq * block_size. */
+pa_status paged_attn_plan(const int32_t* cu_seqlens_q_host, const int32_t* seqlens_k_host,
+                          paged_attn_params* params, size_t* workspace_bytes_needed);
+
+/* Attention forward (see the header comment for layouts).  params must come from
+ * paged_attn_plan with the same lengths the device arrays hold.  total_q == 0
+ * returns PA_OK without a launch.  Rows of sequences with q_b == 0 do not exist
+ * in q/out; no other byte of out is written.  One fused kernel per call, plus a
+ * log-sum-exp combine kernel when params->num_splits > 1. */
+pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_cache,
+                             const float* k_scale, const float* v_scale,
+                             const int32_t* block_table, const int32_t* seqlens_k,
+                             const int32_t* cu_seqlens_q, void* out,
+                             const paged_attn_params* params, void* stream);
+
+/* Zero a workspace (the sticky error word and all scratch).  Call once after
+ * allocating it; asynchronous on stream. */
+pa_status paged_attn_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronise `stream`, read the device error word from `workspace` into *bits
+ * (PA_DEVERR_* flags), and zero it when `clear` is non-zero.  Returns PA_OK when
+ * no bit is set, PA_ERR_BAD_BLOCK_TABLE when PA_DEVERR_BAD_BLOCK is set, and
+ * PA_ERR_DEVICE for any other bit. */
+pa_status paged_attn_read_device_error(void* workspace, int clear, uint32_t* bits, void* stream);
+
+/* INT4 codec (INT4 paged-KV page, Code analysis 2).  pack: int8 values in
+ * [-8, 7], [rows, head_size] -> bytes [rows, head_size/2] with channel 2j in the
+ * low nibble.  unpack: the inverse.  head_size must be even.  A value outside
+ * [-8, 7] is packed from its low 4 bits (the kernel does not check). */
+pa_status paged_kv_pack_int4(const int8_t* src, uint8_t* dst, int64_t rows, int head_size,
+                             void* stream);
+pa_status paged_kv_unpack_int4(const uint8_t* src, int8_t* dst, int64_t rows, int head_size,
+                               void* stream);
+
+/* Test hook: gather the keys (or values) of sequence b, KV head kv through the
+ * block table, decode them with the attention kernel's conversion routines and
+ * store the exact unscaled codes as fp16 (dst_dtype PA_F16) or bf16 (PA_BF16),
+ * contiguous [seqlens_k[b], head_size].  `len_b` is the host value of
+ * seqlens_k[b].  Every code of all three formats is exact in both types. */
+pa_status paged_kv_gather_decode(const void* cache, const int32_t* block_table,
+                                 const paged_attn_params* params, int b, int kv, int len_b,
+                                 int dst_dtype, void* dst, void* stream);
+
+/* Measurement helper: stream `bytes` (multiple of 16, 16-byte aligned) from
+ * `src` with 16-byte loads on every SM and write one 16-byte checksum per block
+ * to `sink` (>= 16 * 148 * 8 bytes).  The read-only HBM ceiling that the
+ * attention kernel is compared against. */
+pa_status paged_attn_stream_read(const void* src, size_t bytes, void* sink, void* stream);
+
+/* Message for the last non-PA_OK status returned on this thread ("" if none). */
+const char* paged_attn_last_error(void);
+
+/* Library version string. */
+const char* paged_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PAGED_ATTN_H */

@@ -1,0 +1,59 @@
+// pa_internal.h -- declarations shared by the host API and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "paged_attn.h"
+
+namespace pa {
+
+// Everything the fused forward kernel needs besides the two tensor maps.
+struct FwdArgs {
+  const void* q;
+  void* out;
+  const float* k_scale;
+  const float* v_scale;
+  const int32_t* block_table;
+  const int32_t* seqlens_k;
+  const int32_t* cu_seqlens_q;
+  float* o_part;    // [num_splits, total_q * H, D] (split mode only)
+  float* lse_part;  // [num_splits, total_q * H] (log2 domain)
+  uint32_t* err;    // sticky device error word
+  int batch, H, Hk, G, maxb, num_blocks, total_q;
+  int q_bf16, out_bf16, causal;
+  int num_row_groups, num_splits, blocks_per_split;
+  float sm_scale_log2;  // softmax_scale * log2(e)
+};
+
+struct CombineArgs {
+  const float* o_part;
+  const float* lse_part;
+  void* out;
+  const int32_t* seqlens_k;
+  const int32_t* cu_seqlens_q;
+  uint32_t* err;
+  int batch, H, Hk, G, D, total_q, num_splits, out_bf16;
+};
+
+// Launchers (pa_attention.cu).  rows_per_cta is 8 or 16.
+cudaError_t launch_forward(int kv_dtype, int head_size, int block_size, int rows_per_cta,
+                           const CUtensorMap& kmap, const CUtensorMap& vmap, const FwdArgs& a,
+                           cudaStream_t stream);
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
+// Shared-memory bytes and threads of one CTA of the forward kernel (for planning/tests).
+int forward_smem_bytes(int kv_dtype, int head_size, int block_size, int rows_per_cta);
+
+// Codec and measurement kernels (pa_codec.cu).
+cudaError_t launch_pack_int4(const int8_t* src, uint8_t* dst, int64_t rows, int head_size,
+                             cudaStream_t s);
+cudaError_t launch_unpack_int4(const uint8_t* src, int8_t* dst, int64_t rows, int head_size,
+                               cudaStream_t s);
+cudaError_t launch_gather_decode(const uint8_t* cache, const int32_t* block_table, int kv_dtype,
+                                 int head_size, int block_size, int kv_num_heads, int maxb,
+                                 int num_blocks, int b, int kv, int len_b, int dst_bf16,
+                                 void* dst, cudaStream_t s);
+cudaError_t launch_stream_read(const void* src, size_t bytes, void* sink, cudaStream_t s);
+
+}  // namespace pa
