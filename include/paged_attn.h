@@ -118,18 +118,25 @@ typedef struct {
   int total_q;            /* cu_seqlens_q[batch] */
   int max_query_len;      /* exact max_b (cu[b+1] - cu[b]) */
   int max_seqlen_k;       /* max_b seqlens_k[b] */
-  int rows_per_cta;       /* query rows (tokens x group heads) per CTA: 8 or 16 */
+  int rows_per_cta;       /* query rows (tokens x group heads) per CTA: 4, 8 or 16
+                             (4: at most 4 rows per sequence and KV head, the fp16
+                             residual of the folded query rides in the idle MMA
+                             columns) */
   int num_row_groups;     /* ceil(max_query_len * H/Hk / rows_per_cta) */
   int num_splits;         /* KV splits of the longest sequence (1 = no split) */
   int blocks_per_split;   /* KV blocks per split */
   size_t workspace_bytes; /* bytes the forward call needs (>= 256) */
   /* ---- supplied by the caller before paged_attn_forward ---- */
   void* workspace;        /* device memory, 256-byte aligned, >= workspace_bytes,
-                             zeroed once with paged_attn_workspace_init */
+                             zeroed once with paged_attn_workspace_init; holds the
+                             error word, the split arrival counters (they return to
+                             zero at the end of every call) and the split partials.
+                             Calls that share a workspace must not overlap on the
+                             GPU. */
   void* profile_events;   /* optional profiling hook: NULL, or a pointer to two
                              cudaEvent_t that paged_attn_forward records on the
                              stream right before and right after the fused
-                             attention kernel (the combine kernel falls outside) */
+                             attention kernel launch */
 } paged_attn_params;
 
 /* Host-side planner.  Validates the problem, computes the exact max_query_len
@@ -145,8 +152,11 @@ pa_status paged_attn_plan(const int32_t* cu_seqlens_q_host, const int32_t* seqle
 /* Attention forward (see the header comment for layouts).  params must come from
  * paged_attn_plan with the same lengths the device arrays hold.  total_q == 0
  * returns PA_OK without a launch.  Rows of sequences with q_b == 0 do not exist
- * in q/out; no other byte of out is written.  One fused kernel per call, plus a
- * log-sum-exp combine kernel when params->num_splits > 1. */
+ * in q/out; no other byte of out is written.  One kernel launch per call; when
+ * params->num_splits > 1 the last CTA of each (sequence, KV head, row group)
+ * merges the split partials (log-sum-exp) inside the same launch.  q, k_scale
+ * and v_scale must be 16-byte aligned, the caches 16-byte aligned, out 4-byte
+ * aligned.  After a device error the workspace should be re-initialised. */
 pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_cache,
                              const float* k_scale, const float* v_scale,
                              const int32_t* block_table, const int32_t* seqlens_k,

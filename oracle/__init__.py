@@ -165,12 +165,13 @@ def lse_combine(o_parts: np.ndarray, lse_parts: np.ndarray) -> np.ndarray:
 
 def gather_decode(w: dict, cache: np.ndarray, b: int, kv: int) -> np.ndarray:
     """Decoded (unscaled) keys of sequence b, head kv, contiguous [L_b, D]."""
-    a = _arrays(w)
+    bt = _c(w["block_table"], np.int32)
+    sk = _c(w["seqlens_k"], np.int32)
     cache = _c(cache, np.uint8)
-    L = int(a["sk"][b])
+    L = int(sk[b])
     out = np.zeros((L, w["head_size"]), dtype=np.float64)
-    rc = _load().oracle_gather_decode(ctypes.byref(_problem(w)), _ptr(cache), _ptr(a["bt"]),
-                                      _ptr(a["sk"]), b, kv, _ptr(out))
+    rc = _load().oracle_gather_decode(ctypes.byref(_problem(w)), _ptr(cache), _ptr(bt),
+                                      _ptr(sk), b, kv, _ptr(out))
     if rc != 0:
         raise ValueError("oracle rejected the gather")
     return out

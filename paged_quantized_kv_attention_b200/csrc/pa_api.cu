@@ -40,9 +40,36 @@ pa_status ok() {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-constexpr size_t kHeaderBytes = 256;   // error word + reserved
-constexpr int kCtasPerSm = 3;          // resident forward CTAs per SM (shared-memory bound)
+constexpr size_t kHeaderBytes = pa::kWsHeaderBytes;  // error word + reserved
+constexpr int kCtasPerSm = 3;          // resident forward CTAs per SM (register bound)
 constexpr int kMinSplitBlocks = 8;     // smallest KV split worth a partial write
+constexpr int kMaxSplits = 128;        // merge weights of one row group fit in shared memory
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Workspace layout shared by the planner and the forward call.
+struct WsLayout {
+  size_t counters, o_part, lse_part, total;
+};
+
+WsLayout ws_layout(const paged_attn_params* p) {
+  WsLayout w;
+  w.counters = kHeaderBytes;
+  size_t off = kHeaderBytes;
+  if (p->num_splits > 1) {
+    const size_t units = static_cast<size_t>(p->batch) * p->kv_num_heads * p->num_row_groups;
+    off = align256(off + units * sizeof(uint32_t));
+    w.o_part = off;
+    const size_t rows = static_cast<size_t>(p->total_q) * p->num_heads;
+    off = align256(off + rows * p->num_splits * p->head_size * sizeof(float));
+    w.lse_part = off;
+    off = align256(off + rows * p->num_splits * sizeof(float));
+  } else {
+    w.o_part = w.lse_part = 0;
+  }
+  w.total = off;
+  return w;
+}
 
 int cache_row_bytes(int kv_dtype, int head_size) {
   return kv_dtype == PA_KV_INT4 ? (head_size + 1) / 2 : head_size;
@@ -178,7 +205,8 @@ pa_status paged_attn_plan(const int32_t* cu_seqlens_q_host, const int32_t* seqle
   p->max_query_len = max_q;
   p->max_seqlen_k = max_k;
   const int64_t max_rows = static_cast<int64_t>(max_q) * G;
-  p->rows_per_cta = max_rows > 8 ? 16 : 8;
+  // 4 rows: decode with G <= 4, fp16 residuals packed into the idle MMA columns
+  p->rows_per_cta = max_rows > 8 ? 16 : (max_rows > 4 ? 8 : 4);
   p->num_row_groups = static_cast<int>((max_rows + p->rows_per_cta - 1) / p->rows_per_cta);
   const int sms = p->num_sms > 0 ? p->num_sms : current_sm_count();
   const int max_nblk = (max_k + bs - 1) / bs;
@@ -196,16 +224,10 @@ pa_status paged_attn_plan(const int32_t* cu_seqlens_q_host, const int32_t* seqle
     }
   }
   if (bps > max_nblk) bps = max_nblk > 0 ? max_nblk : 1;
+  if (max_nblk > 0 && (max_nblk + bps - 1) / bps > kMaxSplits) bps = (max_nblk + kMaxSplits - 1) / kMaxSplits;
   p->blocks_per_split = bps;
   p->num_splits = max_nblk > 0 ? (max_nblk + bps - 1) / bps : 1;
-  size_t ws = kHeaderBytes;
-  if (p->num_splits > 1) {
-    const size_t rows = static_cast<size_t>(total_q) * p->num_heads;
-    ws += rows * p->num_splits * p->head_size * sizeof(float);
-    ws = (ws + 255) & ~static_cast<size_t>(255);
-    ws += rows * p->num_splits * sizeof(float);
-    ws = (ws + 255) & ~static_cast<size_t>(255);
-  }
+  const size_t ws = ws_layout(p).total;
   p->workspace_bytes = ws;
   if (workspace_bytes_needed) *workspace_bytes_needed = ws;
   return ok();
@@ -221,8 +243,12 @@ pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_c
   if (p->total_q < 0 || p->max_query_len < 0)
     return fail(PA_ERR_INVALID_ARG, "params were not filled by paged_attn_plan");
   if (p->total_q == 0 || p->batch == 0 || p->max_query_len == 0) return ok();
-  if (p->rows_per_cta != 8 && p->rows_per_cta != 16)
+  if (p->rows_per_cta != 4 && p->rows_per_cta != 8 && p->rows_per_cta != 16)
     return fail(PA_ERR_INVALID_ARG, "params were not filled by paged_attn_plan (rows_per_cta)");
+  if (p->rows_per_cta == 4 && p->max_query_len * (p->num_heads / p->kv_num_heads) > 4)
+    return fail(PA_ERR_INVALID_ARG, "params were not filled by paged_attn_plan (rows_per_cta)");
+  if (p->num_splits > kMaxSplits)
+    return fail(PA_ERR_INVALID_ARG, "num_splits %d exceeds %d", p->num_splits, kMaxSplits);
   const int G = p->num_heads / p->kv_num_heads;
   const int64_t need_rg = (static_cast<int64_t>(p->max_query_len) * G + p->rows_per_cta - 1) /
                           p->rows_per_cta;
@@ -236,8 +262,9 @@ pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_c
     return fail(PA_ERR_INVALID_ARG, "a device pointer argument is NULL");
   if (!aligned(k_cache, 16) || !aligned(v_cache, 16))
     return fail(PA_ERR_INVALID_ARG, "k_cache/v_cache must be 16-byte aligned (TMA)");
-  if (!aligned(q, 4) || !aligned(out, 4) || !aligned(k_scale, 4) || !aligned(v_scale, 4))
-    return fail(PA_ERR_INVALID_ARG, "q/out/scales must be 4-byte aligned");
+  if (!aligned(q, 16) || !aligned(k_scale, 16) || !aligned(v_scale, 16))
+    return fail(PA_ERR_INVALID_ARG, "q, k_scale and v_scale must be 16-byte aligned (bulk copies)");
+  if (!aligned(out, 4)) return fail(PA_ERR_INVALID_ARG, "out must be 4-byte aligned");
   if (p->workspace == nullptr || p->workspace_bytes < kHeaderBytes)
     return fail(PA_ERR_WORKSPACE, "workspace missing (plan asks for %zu bytes)",
                 p->workspace_bytes);
@@ -249,6 +276,10 @@ pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_c
   if ((st = encode_cache_map(v_cache, p, &vmap)) != PA_OK) return st;
 
   uint8_t* ws = static_cast<uint8_t*>(p->workspace);
+  const WsLayout lay = ws_layout(p);
+  if (lay.total > p->workspace_bytes)
+    return fail(PA_ERR_WORKSPACE, "workspace_bytes %zu < %zu needed for %d splits",
+                p->workspace_bytes, lay.total, p->num_splits);
   pa::FwdArgs a;
   a.q = q;
   a.out = out;
@@ -258,21 +289,9 @@ pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_c
   a.seqlens_k = seqlens_k;
   a.cu_seqlens_q = cu_seqlens_q;
   a.err = reinterpret_cast<uint32_t*>(ws);
-  a.o_part = nullptr;
-  a.lse_part = nullptr;
-  const size_t rows = static_cast<size_t>(p->total_q) * p->num_heads;
-  if (p->num_splits > 1) {
-    size_t off = kHeaderBytes;
-    a.o_part = reinterpret_cast<float*>(ws + off);
-    off += rows * p->num_splits * p->head_size * sizeof(float);
-    off = (off + 255) & ~static_cast<size_t>(255);
-    a.lse_part = reinterpret_cast<float*>(ws + off);
-    off += rows * p->num_splits * sizeof(float);
-    off = (off + 255) & ~static_cast<size_t>(255);
-    if (off > p->workspace_bytes)
-      return fail(PA_ERR_WORKSPACE, "workspace_bytes %zu < %zu needed for %d splits",
-                  p->workspace_bytes, off, p->num_splits);
-  }
+  a.counters = reinterpret_cast<uint32_t*>(ws + lay.counters);
+  a.o_part = p->num_splits > 1 ? reinterpret_cast<float*>(ws + lay.o_part) : nullptr;
+  a.lse_part = p->num_splits > 1 ? reinterpret_cast<float*>(ws + lay.lse_part) : nullptr;
   a.batch = p->batch;
   a.H = p->num_heads;
   a.Hk = p->kv_num_heads;
@@ -300,25 +319,6 @@ pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_c
   if (e != cudaSuccess) return cuda_status(e, "forward launch");
   if (ev != nullptr && (e = cudaEventRecord(ev[1], s)) != cudaSuccess)
     return cuda_status(e, "profile event record");
-  if (p->num_splits > 1) {
-    pa::CombineArgs c;
-    c.o_part = a.o_part;
-    c.lse_part = a.lse_part;
-    c.out = out;
-    c.seqlens_k = seqlens_k;
-    c.cu_seqlens_q = cu_seqlens_q;
-    c.err = a.err;
-    c.batch = p->batch;
-    c.H = p->num_heads;
-    c.Hk = p->kv_num_heads;
-    c.G = G;
-    c.D = p->head_size;
-    c.total_q = p->total_q;
-    c.num_splits = p->num_splits;
-    c.out_bf16 = a.out_bf16;
-    e = pa::launch_combine(c, s);
-    if (e != cudaSuccess) return cuda_status(e, "combine launch");
-  }
   return ok();
 }
 

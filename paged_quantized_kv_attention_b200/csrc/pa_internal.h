@@ -18,31 +18,26 @@ struct FwdArgs {
   const int32_t* block_table;
   const int32_t* seqlens_k;
   const int32_t* cu_seqlens_q;
-  float* o_part;    // [num_splits, total_q * H, D] (split mode only)
-  float* lse_part;  // [num_splits, total_q * H] (log2 domain)
-  uint32_t* err;    // sticky device error word
+  float* o_part;        // [num_splits, total_q * H, D] (split mode only)
+  float* lse_part;      // [num_splits, total_q * H] (log2 domain)
+  uint32_t* counters;   // [batch * Hk * num_row_groups] split arrival counters (self-resetting)
+  uint32_t* err;        // sticky device error word
   int batch, H, Hk, G, maxb, num_blocks, total_q;
   int q_bf16, out_bf16, causal;
   int num_row_groups, num_splits, blocks_per_split;
   float sm_scale_log2;  // softmax_scale * log2(e)
 };
 
-struct CombineArgs {
-  const float* o_part;
-  const float* lse_part;
-  void* out;
-  const int32_t* seqlens_k;
-  const int32_t* cu_seqlens_q;
-  uint32_t* err;
-  int batch, H, Hk, G, D, total_q, num_splits, out_bf16;
-};
+// Workspace layout: [0, 256) error word; [256, 256 + counters) split counters;
+// then the partial outputs and their log-sum-exps (256-byte aligned each).
+constexpr size_t kWsHeaderBytes = 256;
 
-// Launchers (pa_attention.cu).  rows_per_cta is 8 or 16.
+// Launcher (pa_attention.cu).  rows_per_cta is 4 (decode rows packed with their
+// fp16 residuals), 8 or 16.
 cudaError_t launch_forward(int kv_dtype, int head_size, int block_size, int rows_per_cta,
                            const CUtensorMap& kmap, const CUtensorMap& vmap, const FwdArgs& a,
                            cudaStream_t stream);
-cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
-// Shared-memory bytes and threads of one CTA of the forward kernel (for planning/tests).
+// Dynamic shared memory of one forward CTA (-1 for an unsupported combination).
 int forward_smem_bytes(int kv_dtype, int head_size, int block_size, int rows_per_cta);
 
 // Codec and measurement kernels (pa_codec.cu).

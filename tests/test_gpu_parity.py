@@ -200,7 +200,8 @@ def test_bad_block_id_is_flagged_not_faulted():
     ov["block_table"] = prob["block_table"]
     ref = oracle.paged_attn(ov)
     got = out.double().cpu().numpy()
-    assert np.max(np.abs(got[0] - ref[0])) <= _gpu.TOL[0] * _gpu.vmax(w, [0])
+    vm = _gpu.vmax(dict(w, block_table=prob["block_table"]), [0])
+    assert np.max(np.abs(got[0] - ref[0])) <= _gpu.TOL[0] * vm
 
 
 def test_non_finite_k_scale_is_flagged():
