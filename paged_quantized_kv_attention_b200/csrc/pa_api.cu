@@ -41,8 +41,9 @@ pa_status ok() {
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 constexpr size_t kHeaderBytes = pa::kWsHeaderBytes;  // error word + reserved
-constexpr int kCtasPerSm = 3;          // resident forward CTAs per SM (register bound)
-constexpr int kMinSplitBlocks = 8;     // smallest KV split worth a partial write
+constexpr int kCtasPerSm = 3;          // typical resident forward CTAs per SM
+constexpr int kItemsPerCta = 4;        // work items per resident CTA wanted for balance
+constexpr int64_t kMinSplitBytes = 64 << 10;  // smallest KV split worth a partial write
 constexpr int kMaxSplits = 128;        // merge weights of one row group fit in shared memory
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -214,13 +215,18 @@ pa_status paged_attn_plan(const int32_t* cu_seqlens_q_host, const int32_t* seqle
   if (p->split_blocks > 0) {
     bps = p->split_blocks;
   } else if (p->split_blocks == 0) {
+    // Split the KV of a unit (flash decoding) when the units alone would leave
+    // the persistent CTAs with fewer than kItemsPerCta items each; splits carry
+    // at least kMinSplitBytes of K+V so the partial write stays small.
     const int64_t units = static_cast<int64_t>(B) * p->kv_num_heads * p->num_row_groups;
-    const int64_t slots = static_cast<int64_t>(sms) * kCtasPerSm;
-    if (units > 0 && units < slots && max_nblk > kMinSplitBlocks) {
+    const int64_t want_items = static_cast<int64_t>(sms) * kCtasPerSm * kItemsPerCta;
+    const int64_t block_bytes = 2LL * bs * cache_row_bytes(p->kv_dtype, p->head_size);
+    const int64_t min_bps = (kMinSplitBytes + block_bytes - 1) / block_bytes;
+    if (units > 0 && units < want_items && max_nblk > min_bps) {
       const int64_t work = total_blocks * p->kv_num_heads * p->num_row_groups;
-      int64_t want = (work + slots - 1) / slots;
-      if (want < kMinSplitBlocks) want = kMinSplitBlocks;
-      bps = static_cast<int>(want);
+      int64_t b2 = (work + want_items - 1) / want_items;
+      if (b2 < min_bps) b2 = min_bps;
+      bps = static_cast<int>(b2);
     }
   }
   if (bps > max_nblk) bps = max_nblk > 0 ? max_nblk : 1;
@@ -290,6 +296,7 @@ pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_c
   a.cu_seqlens_q = cu_seqlens_q;
   a.err = reinterpret_cast<uint32_t*>(ws);
   a.counters = reinterpret_cast<uint32_t*>(ws + lay.counters);
+  a.work = reinterpret_cast<uint32_t*>(ws + pa::kWsWorkOffset);
   a.o_part = p->num_splits > 1 ? reinterpret_cast<float*>(ws + lay.o_part) : nullptr;
   a.lse_part = p->num_splits > 1 ? reinterpret_cast<float*>(ws + lay.lse_part) : nullptr;
   a.batch = p->batch;
@@ -305,6 +312,11 @@ pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_c
   a.num_row_groups = p->num_row_groups;
   a.num_splits = p->num_splits;
   a.blocks_per_split = p->blocks_per_split;
+  const int64_t items = static_cast<int64_t>(p->batch) * p->kv_num_heads * p->num_row_groups *
+                        p->num_splits;
+  if (items >= (int64_t(1) << 31)) return fail(PA_ERR_UNSUPPORTED, "too many work items");
+  a.num_items = static_cast<int>(items);
+  a.num_sms = p->num_sms > 0 ? p->num_sms : current_sm_count();
   const float scale = p->softmax_scale > 0.f ? p->softmax_scale
                                              : 1.0f / sqrtf(static_cast<float>(p->head_size));
   a.sm_scale_log2 = scale * 1.4426950408889634f;

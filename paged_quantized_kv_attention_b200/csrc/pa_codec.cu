@@ -54,7 +54,8 @@ __device__ __forceinline__ void decode_word(uint32_t x, uint16_t* h, int& n) {
     h[0] = p01 & 0xFFFF; h[1] = p01 >> 16; h[2] = p23 & 0xFFFF; h[3] = p23 >> 16;
     n = 4;
   } else if constexpr (KV == PA_KV_FP8_E4M3) {
-    const uint32_t p01 = e4m3x2_to_h2(x), p23 = e4m3x2_to_h2(x >> 16);
+    uint32_t p01, p23;
+    e4m3x4_to_h2x2(x, p01, p23);
     h[0] = p01 & 0xFFFF; h[1] = p01 >> 16; h[2] = p23 & 0xFFFF; h[3] = p23 >> 16;
     n = 4;
   } else {

@@ -63,11 +63,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait that lets the hardware suspend the thread for up to hint_ns while the
+// phase is incomplete (it resumes as soon as the phase completes).
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity,
+                                                      uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+constexpr uint32_t kSuspendHintNs = 20000;
+
 // Wait for the phase with the given parity to complete, for at most kWaitLimitNs.
+// The thread sleeps in try_wait; the clock is read only after a failed suspend.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_suspend(bar, parity, kSuspendHintNs)) {
     if (global_timer_ns() - t0 > kWaitLimitNs) return false;
   }
   return true;
@@ -76,7 +94,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
 // Same, against an absolute deadline shared by several waits.
 __device__ __forceinline__ bool mbar_wait_until(uint32_t bar, uint32_t parity,
                                                 uint64_t deadline_ns) {
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_suspend(bar, parity, kSuspendHintNs)) {
     if (global_timer_ns() > deadline_ns) return false;
   }
   return true;
@@ -174,11 +192,44 @@ __device__ __forceinline__ uint32_t i4hi_to_h2(uint32_t x) {
   return h22u(__hfma2(u2h2(h), u2h2(0x2C002C00u), u2h2(0xD480D480u)));  // 1/16, -72
 }
 
-// FP8 e4m3, two codes in the low 16 bits of x -> fp16x2 (low code -> low half).
-__device__ __forceinline__ uint32_t e4m3x2_to_h2(uint32_t x) {
-  const __half2_raw r = __nv_cvt_fp8x2_to_halfraw2(
-      static_cast<__nv_fp8x2_storage_t>(x & 0xFFFFu), __NV_E4M3);
-  return static_cast<uint32_t>(r.x) | (static_cast<uint32_t>(r.y) << 16);
+// FP8 e4m3: the four codes of x -> two fp16x2 (bytes 0,1 -> lo; bytes 2,3 -> hi;
+// the lower code of each pair lands in the lower half).
+__device__ __forceinline__ void e4m3x4_to_h2x2(uint32_t x, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(x));
+}
+
+// INT4 -> u8 (code + 8) bytes: nibbles 0,2,4,6 of x (low nibble of each byte).
+__device__ __forceinline__ uint32_t i4lo_to_u8x4(uint32_t x) { return (x & 0x0F0F0F0Fu) ^ 0x08080808u; }
+// nibbles 1,3,5,7 of x (high nibble of each byte).
+__device__ __forceinline__ uint32_t i4hi_to_u8x4(uint32_t x) {
+  return ((x >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+}
+
+// D = A(16x32, row) * B(32x8, col) + D with int8 operands and int32 accumulators;
+// A is signed (s8) or unsigned (u8), B signed.
+template <bool A_UNSIGNED>
+__device__ __forceinline__ void imma_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                           uint32_t a3, uint32_t b0, uint32_t b1) {
+  if constexpr (A_UNSIGNED) {
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  } else {
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  }
+}
+
+// Exact int -> float for |v| < 2^22 with an integer offset folded in:
+// returns (float)(v - off) using the 1.5 * 2^23 magic number.
+__device__ __forceinline__ float int_to_float_exact(int v, int magic_minus_off) {
+  return __int_as_float(v + magic_minus_off) - 12582912.0f;
 }
 
 __device__ __forceinline__ uint32_t pack_f32x2_to_h2(float lo, float hi) {

@@ -21,16 +21,21 @@ struct FwdArgs {
   float* o_part;        // [num_splits, total_q * H, D] (split mode only)
   float* lse_part;      // [num_splits, total_q * H] (log2 domain)
   uint32_t* counters;   // [batch * Hk * num_row_groups] split arrival counters (self-resetting)
+  uint32_t* work;       // [2]: next work item, CTAs finished (both rewound by the last CTA)
   uint32_t* err;        // sticky device error word
   int batch, H, Hk, G, maxb, num_blocks, total_q;
   int q_bf16, out_bf16, causal;
   int num_row_groups, num_splits, blocks_per_split;
+  int num_items;        // batch * Hk * num_row_groups * num_splits
+  int num_sms;          // SMs of the device (grid = resident CTAs per SM x num_sms)
   float sm_scale_log2;  // softmax_scale * log2(e)
 };
 
-// Workspace layout: [0, 256) error word; [256, 256 + counters) split counters;
-// then the partial outputs and their log-sum-exps (256-byte aligned each).
+// Workspace layout: [0, 256) header: error word at byte 0, work counters at
+// byte 64; then the split counters; then the partial outputs and their
+// log-sum-exps (256-byte aligned each).
 constexpr size_t kWsHeaderBytes = 256;
+constexpr size_t kWsWorkOffset = 64;
 
 // Launcher (pa_attention.cu).  rows_per_cta is 4 (decode rows packed with their
 // fp16 residuals), 8 or 16.

@@ -241,3 +241,29 @@ def test_parity_full_size_sampled(name):
     assert np.all(np.isfinite(got))
     st, bits = pa.paged_attn_read_device_error(ws)
     assert st == pa.PA_OK and bits == 0
+
+
+def test_repeated_calls_share_one_workspace():
+    """Work and split counters rewind at the end of every call: back-to-back calls
+    on one workspace (persistent CTAs, many split items, shallow stage rings)
+    give bit-identical, oracle-checked results."""
+    w = workloads.shrink("c3_int8_long_split", 21, max_len=6000, batch=3)
+    d = _gpu.to_device(w)
+    p, ws_bytes = _gpu.plan(w, split_blocks=4)
+    assert p.num_splits > 8
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    pa.paged_attn_workspace_init(ws, ws_bytes)
+    p.workspace = ws.data_ptr()
+    outs = []
+    for _ in range(4):
+        out = torch.empty((int(w["cu_seqlens_q"][-1]), w["num_heads"], w["head_size"]),
+                          dtype=torch.bfloat16, device="cuda")
+        pa.paged_attn_forward(d["q"], d["k_cache"], d["v_cache"], d["k_scale"], d["v_scale"],
+                              d["block_table"], d["seqlens_k"], d["cu_seqlens_q"], out, p)
+        outs.append(out)
+    torch.cuda.synchronize()
+    st, bits = pa.paged_attn_read_device_error(ws)
+    assert st == pa.PA_OK and bits == 0
+    for o in outs[1:]:
+        assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
+    _check(w, outs[-1])

@@ -70,9 +70,11 @@ def test_plan_zero_new_tokens_everywhere_is_a_no_op():
 @pytest.mark.parametrize("name,split", [("c1_tiny_int8", False), ("c2_int4_decode", True),
                                         ("c3_int8_long_split", True),
                                         ("c4_ragged_prefill_int8", False),
-                                        ("c5_fp8_large_batch", False)])
+                                        ("c5_fp8_large_batch", True)])
 def test_plan_split_decisions_on_the_workload_shapes(name, split):
-    """Flash-decoding split only when B*Hk*row groups underfills 148 SMs x 3 CTAs."""
+    """Flash-decoding split only when the units (B * Hk * row groups) give the
+    persistent CTAs (148 SMs x 3) fewer than 4 work items each, in splits of at
+    least 64 KB of K+V."""
     rng = np.random.default_rng(0)
     if name == "c1_tiny_int8":
         B, H, Hk, D, bs, L, ql = 2, 4, 1, 64, 16, np.array([37, 64]), np.ones(2, int)
@@ -89,15 +91,17 @@ def test_plan_split_decisions_on_the_workload_shapes(name, split):
         B, H, Hk, D, bs, L, ql = 128, 64, 8, 128, 16, np.full(128, 8192), np.ones(128, int)
     cu = np.concatenate([[0], np.cumsum(ql)]).astype(np.int32)
     maxb = int(-(-L.max() // bs))
+    kvd = pa.PA_KV_INT4 if name == "c2_int4_decode" else pa.PA_KV_INT8
     p = _params(batch=B, num_heads=H, kv_num_heads=Hk, head_size=D, block_size=bs,
-                num_blocks=maxb * B, max_blocks_per_seq=maxb)
+                num_blocks=maxb * B, max_blocks_per_seq=maxb, kv_dtype=kvd)
     ws = pa.paged_attn_plan(cu, L, p)
     assert (p.num_splits > 1) == split
     assert p.num_splits * p.blocks_per_split >= -(-int(L.max()) // bs)
     assert ws >= 256 and ws % 256 == 0
     if split:
         assert ws >= 256 + p.num_splits * p.total_q * H * (D + 1) * 4
-        assert p.blocks_per_split >= 8
+        chs = D // 2 if name == "c2_int4_decode" else D
+        assert p.blocks_per_split * 2 * bs * chs >= 64 * 1024
 
 
 def test_plan_forced_and_disabled_split():
