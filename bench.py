@@ -1,9 +1,10 @@
 #!/usr/bin/env python
 """Benchmark of paged quantised-KV attention on B200 (one JSON line on rank 0).
 
-A step is one call of the whole hot path (fused attention kernel, plus the
-log-sum-exp combine kernel when the planner splits the KV) over one batch of
-seeded synthetic input whose cache is already resident in HBM.  Between steps
+A step is one call of the whole hot path (one fused kernel launch; when the
+planner splits the KV, the last split of each unit merges the partials by
+log-sum-exp inside the same launch) over one batch of seeded synthetic input
+whose cache is already resident in HBM.  Between steps
 the L2 cache (126 MB) is flushed by writing a 256 MB buffer, outside the timed
 spans; each step is timed with CUDA events on the launching stream.
 
@@ -70,17 +71,20 @@ def kernel_source_sha() -> str:
 
 
 def ncu_traffic(name: str):
-    """DRAM bytes per launch from the committed ncu summary, if it still matches
-    the kernel source (else None)."""
-    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    """DRAM bytes (read + write) per launch of the fused kernel from the committed
+    ncu summary profiles/ncu_traffic.txt, if it was taken on the current kernel
+    source (else None).  Line format: workload kernel_source_sha bytes_per_launch."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
     try:
         with open(path) as f:
-            rec = json.load(f).get(name)
+            for ln in f:
+                parts = ln.split()
+                if len(parts) >= 3 and not ln.startswith("#") and parts[0] == name:
+                    if parts[1] == kernel_source_sha():
+                        return int(parts[2])
     except (OSError, ValueError):
         return None
-    if not rec or rec.get("kernel_source_sha") != kernel_source_sha():
-        return None
-    return rec.get("dram_bytes_per_launch")
+    return None
 
 
 def measured_peaks():
@@ -287,7 +291,7 @@ def measure(name: str, steps: int, warmup: int, dev: str, flush, with_e2e: bool)
     res = dict(w=w, ab=ab, p=p, call_ms=call, kern_ms=kern,
                value=ab["total"] / (call * 1e-3) / 1e9,
                kernel_gbs=ab["fwd"] / (kern * 1e-3) / 1e9, peak=peak, peak_kind=peak_kind,
-               launches_per_step=1 + (1 if p.num_splits > 1 else 0))
+               launches_per_step=1)
     if with_e2e:
         e2e_ms, h2d, d2h = time_e2e(w, d, p, max(5, steps // 2), 2, flush)
         res["e2e"] = dict(value=ab["total"] / (statistics.mean(e2e_ms) * 1e-3) / 1e9,
