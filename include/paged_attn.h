@@ -163,6 +163,43 @@ pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_c
                              const int32_t* cu_seqlens_q, void* out,
                              const paged_attn_params* params, void* stream);
 
+/* Size of the library-owned scratch used by paged_attn_forward_noalloc: 16 MiB,
+ * held by every GPU that loads the library until the process exits. */
+#define PA_NOALLOC_MAX_WORKSPACE_BYTES (16u << 20)
+
+/* paged_attn_forward for callers that cannot allocate device memory.  (The
+ * pages have no counterpart: this entry point exists for the caller's memory
+ * model, not for the method.)
+ *
+ * Who needs it: code that must not call cudaMalloc or any allocator where it
+ * runs attention -- an operator inside a host framework that owns every device
+ * buffer, a fixed memory plan replayed step after step, a real-time loop whose
+ * memory is frozen at start-up.  Such callers hold q, the caches, the scales,
+ * the block table, the lengths and out, but have no workspace to give.
+ *
+ * What it does: the same computation and kernel launch as paged_attn_forward
+ * (same arguments, layouts and results), with the workspace taken from a
+ * library-owned device array of PA_NOALLOC_MAX_WORKSPACE_BYTES instead of
+ * params->workspace (which is ignored).  It allocates and frees nothing.
+ *  - params must come from paged_attn_plan; if its workspace_bytes exceeds
+ *    PA_NOALLOC_MAX_WORKSPACE_BYTES the call returns PA_ERR_WORKSPACE before any
+ *    device work (plan again with a larger split_blocks, i.e. fewer splits, or
+ *    use paged_attn_forward with your own workspace).
+ *  - The first call on a device looks up the array's device address on that
+ *    device (cudaGetSymbolAddress, the device current); make that first call
+ *    before any stream capture on the device.
+ *  - Every call clears the array's error word and counters on `stream`
+ *    (cudaMemsetAsync) before the launch; the array keeps the rest of the last
+ *    call's contents.  There is no device-error readback for this path.
+ *  - All calls in the process share the one array per device: calls whose
+ *    executions overlap on the GPU (different streams without ordering between
+ *    them) race on it and give wrong results.  Order them on one stream. */
+pa_status paged_attn_forward_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                     const float* k_scale, const float* v_scale,
+                                     const int32_t* block_table, const int32_t* seqlens_k,
+                                     const int32_t* cu_seqlens_q, void* out,
+                                     const paged_attn_params* params, void* stream);
+
 /* Zero a workspace (the sticky error word and all scratch).  Call once after
  * allocating it; asynchronous on stream. */
 pa_status paged_attn_workspace_init(void* workspace, size_t workspace_bytes, void* stream);

@@ -21,8 +21,10 @@ PA_ERR_BAD_BLOCK_TABLE, PA_ERR_CUDA, PA_ERR_DEVICE = -4, -5, -6
 PA_KV_INT8, PA_KV_INT4, PA_KV_FP8_E4M3 = 0, 1, 2
 PA_F16, PA_BF16 = 0, 1
 PA_DEVERR_BAD_BLOCK, PA_DEVERR_TIMEOUT, PA_DEVERR_BAD_SCALE, PA_DEVERR_BAD_LENGTH = 1, 2, 4, 8
+PA_NOALLOC_MAX_WORKSPACE_BYTES = 16 << 20
 
-EXPORTED = ["paged_attn_plan", "paged_attn_forward", "paged_attn_workspace_init",
+EXPORTED = ["paged_attn_plan", "paged_attn_forward", "paged_attn_forward_noalloc",
+            "paged_attn_workspace_init",
             "paged_attn_read_device_error", "paged_kv_pack_int4", "paged_kv_unpack_int4",
             "paged_kv_gather_decode", "paged_attn_stream_read", "paged_attn_last_error",
             "paged_attn_version"]
@@ -64,6 +66,7 @@ def lib() -> ctypes.CDLL:
         PP = ctypes.POINTER(paged_attn_params)
         L.paged_attn_plan.argtypes = [P, P, PP, ctypes.POINTER(ctypes.c_size_t)]
         L.paged_attn_forward.argtypes = [P] * 9 + [PP, P]
+        L.paged_attn_forward_noalloc.argtypes = [P] * 9 + [PP, P]
         L.paged_attn_workspace_init.argtypes = [P, S, P]
         L.paged_attn_read_device_error.argtypes = [P, I, ctypes.POINTER(ctypes.c_uint32), P]
         L.paged_kv_pack_int4.argtypes = [P, P, ctypes.c_int64, I, P]
@@ -125,6 +128,17 @@ def paged_attn_forward(q, k_cache, v_cache, k_scale, v_scale, block_table, seqle
                                     _ptr(v_scale), _ptr(block_table), _ptr(seqlens_k),
                                     _ptr(cu_seqlens_q), _ptr(out), ctypes.byref(params),
                                     _stream(stream)))
+
+
+def paged_attn_forward_noalloc(q, k_cache, v_cache, k_scale, v_scale, block_table, seqlens_k,
+                               cu_seqlens_q, out, params: paged_attn_params, stream=None):
+    """paged_attn_forward without a caller workspace: the library's own static
+    device scratch (PA_NOALLOC_MAX_WORKSPACE_BYTES) is used instead, for callers
+    that cannot allocate device memory.  params.workspace is ignored."""
+    _check(lib().paged_attn_forward_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale),
+                                            _ptr(v_scale), _ptr(block_table), _ptr(seqlens_k),
+                                            _ptr(cu_seqlens_q), _ptr(out), ctypes.byref(params),
+                                            _stream(stream)))
 
 
 def paged_attn_workspace_init(workspace, nbytes: int, stream=None):

@@ -170,6 +170,11 @@ pa_status cuda_status(cudaError_t e, const char* what) {
 
 }  // namespace
 
+pa_status pa::set_last_error(pa_status st, const char* msg) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s", msg);
+  return st;
+}
+
 extern "C" {
 
 const char* paged_attn_last_error(void) { return g_last_error; }

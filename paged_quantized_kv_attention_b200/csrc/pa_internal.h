@@ -45,6 +45,10 @@ cudaError_t launch_forward(int kv_dtype, int head_size, int block_size, int rows
 // Dynamic shared memory of one forward CTA (-1 for an unsupported combination).
 int forward_smem_bytes(int kv_dtype, int head_size, int block_size, int rows_per_cta);
 
+// Sets the thread's message for paged_attn_last_error() and returns st
+// (pa_api.cu; used by entry points defined in other files).
+pa_status set_last_error(pa_status st, const char* msg);
+
 // Codec and measurement kernels (pa_codec.cu).
 cudaError_t launch_pack_int4(const int8_t* src, uint8_t* dst, int64_t rows, int head_size,
                              cudaStream_t s);

@@ -189,3 +189,25 @@ def test_workload_generators_follow_the_stated_shapes():
     k = w["k_cache"].view(np.int8)
     assert k.min() >= -127 and k.max() <= 127
     assert w["k_scale"].min() >= 0.005 and w["k_scale"].max() <= 0.02
+
+
+def test_noalloc_rejects_plans_beyond_its_static_scratch():
+    """The no-alloc forward refuses, before any device work, a plan whose
+    workspace exceeds the library's static scratch."""
+    B, ql, L = 8, 16, 4096
+    cu = np.arange(0, B * ql + 1, ql, dtype=np.int32)
+    p = _params(batch=B, num_heads=64, kv_num_heads=8, max_blocks_per_seq=L // 16,
+                num_blocks=B * L // 16, split_blocks=8)
+    need = pa.paged_attn_plan(cu, np.full(B, L, dtype=np.int32), p)
+    assert need > pa.PA_NOALLOC_MAX_WORKSPACE_BYTES
+    fake = np.zeros(64, dtype=np.uint8)  # host memory: never dereferenced
+    with pytest.raises(pa.PagedAttnError) as ei:
+        pa.paged_attn_forward_noalloc(*([fake] * 9), p, stream=0)
+    assert ei.value.status == pa.PA_ERR_WORKSPACE
+    assert "static scratch" in pa.paged_attn_last_error()
+    unplanned = pa.make_params(batch=1, num_heads=8, kv_num_heads=8, head_size=128,
+                               block_size=16, num_blocks=4, max_blocks_per_seq=4,
+                               kv_dtype=pa.PA_KV_INT8, q_dtype=pa.PA_F16, out_dtype=pa.PA_F16)
+    with pytest.raises(pa.PagedAttnError) as ei:
+        pa.paged_attn_forward_noalloc(*([fake] * 9), unplanned, stream=0)
+    assert ei.value.status == pa.PA_ERR_INVALID_ARG
