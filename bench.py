@@ -4,9 +4,12 @@
 A step is one call of the whole hot path (one fused kernel launch; when the
 planner splits the KV, the last split of each unit merges the partials by
 log-sum-exp inside the same launch) over one batch of seeded synthetic input
-whose cache is already resident in HBM.  Between steps
-the L2 cache (126 MB) is flushed by writing a 256 MB buffer, outside the timed
-spans; each step is timed with CUDA events on the launching stream.
+whose cache is already resident in HBM.  Consecutive steps read different
+copies ("replicas") of the whole input set, rotating through enough of them that
+the bytes read between two uses of one copy exceed three times the 126 MB L2, so
+every step reads its KV cache from HBM; a workload too small for that (the tiny
+case) instead flushes L2 by writing a 256 MB buffer before each step, outside the
+timed span.  Each step is timed with CUDA events on the launching stream.
 
 Headline workload (N=1): INT4 packed decode, B=16, q_len=1, 32 query / 8 KV
 heads, head_size 128, block_size 16, seqlens_k ~ U[512, 4096].  The other
@@ -42,6 +45,8 @@ import workloads  # noqa: E402
 HEADLINE = "c2_int4_decode"
 EXTRA = ["c3_int8_long_split", "c5_fp8_large_batch", "c4_ragged_prefill_int8", "c1_tiny_int8"]
 L2_FLUSH_BYTES = 256 << 20
+L2_BYTES = 126 << 20
+MAX_REPLICAS = 16
 SPIN_CYCLES = 200000  # ~0.1 ms of GPU work queued ahead of every timed span
 
 
@@ -146,14 +151,22 @@ class ClockSampler:
                 "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
 
 
-def setup(w: dict, dev: str):
+def setup(w: dict, dev: str, replicas: int = 1):
+    """Device copies of the workload: a list of `replicas` independent input sets
+    (each with its own output), one plan and one workspace shared by all."""
     import paged_quantized_kv_attention_b200 as pa
     from_np = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)  # noqa: E731
-    d = dict(q=w["q"].to(dev), k_cache=from_np(w["k_cache"]), v_cache=from_np(w["v_cache"]),
-             k_scale=from_np(w["k_scale"].astype(np.float32)),
-             v_scale=from_np(w["v_scale"].astype(np.float32)),
-             block_table=from_np(w["block_table"]), seqlens_k=from_np(w["seqlens_k"]),
-             cu_seqlens_q=from_np(w["cu_seqlens_q"]))
+    odt = torch.bfloat16 if w["out_dtype"] == 1 else torch.float16
+    T = int(w["cu_seqlens_q"][-1])
+    reps = []
+    for _ in range(replicas):
+        d = dict(q=w["q"].to(dev), k_cache=from_np(w["k_cache"]), v_cache=from_np(w["v_cache"]),
+                 k_scale=from_np(w["k_scale"].astype(np.float32)),
+                 v_scale=from_np(w["v_scale"].astype(np.float32)),
+                 block_table=from_np(w["block_table"]), seqlens_k=from_np(w["seqlens_k"]),
+                 cu_seqlens_q=from_np(w["cu_seqlens_q"]))
+        d["out"] = torch.empty((T, w["num_heads"], w["head_size"]), dtype=odt, device=dev)
+        reps.append(d)
     p = pa.make_params(batch=w["batch"], num_heads=w["num_heads"], kv_num_heads=w["kv_num_heads"],
                        head_size=w["head_size"], block_size=w["block_size"],
                        num_blocks=w["num_blocks"], max_blocks_per_seq=w["max_blocks_per_seq"],
@@ -163,11 +176,27 @@ def setup(w: dict, dev: str):
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     pa.paged_attn_workspace_init(ws, ws_bytes)
     p.workspace = ws.data_ptr()
-    odt = torch.bfloat16 if w["out_dtype"] == 1 else torch.float16
-    T = int(w["cu_seqlens_q"][-1])
-    d["out"] = torch.empty((T, w["num_heads"], w["head_size"]), dtype=odt, device=dev)
-    d["ws"] = ws
-    return d, p
+    for d in reps:
+        d["ws"] = ws
+    return reps, p
+
+
+def l2_plan(w: dict):
+    """(replicas, flush): rotate replicas so that > 3 x L2 bytes are read between
+    two uses of one copy; fall back to flushing when that needs too many copies."""
+    foot = algorithmic_bytes(w)["total"]
+    need = -(-3 * L2_BYTES // max(foot, 1))
+    if need <= MAX_REPLICAS:
+        return max(1, int(need)), False
+    return 1, True
+
+
+def l2_desc(replicas: int, flush: bool, w: dict) -> str:
+    if flush:
+        return "flushed before every step (256 MB write, outside the timed span)"
+    foot = algorithmic_bytes(w)["total"] / 1e6
+    return ("inputs larger than L2: %d rotating replica(s) of the whole input set, %.0f MB read "
+            "per step, %.0f MB between two uses of one copy" % (replicas, foot, foot * replicas))
 
 
 def _event_handles(evs):
@@ -176,17 +205,23 @@ def _event_handles(evs):
     return arr
 
 
-def time_device(w, d, p, steps, warmup, flush):
-    """Per-step device time of the whole call and of the fused kernel (ms lists)."""
+def _args(d):
+    return (d["q"], d["k_cache"], d["v_cache"], d["k_scale"], d["v_scale"], d["block_table"],
+            d["seqlens_k"], d["cu_seqlens_q"], d["out"])
+
+
+def time_device(w, reps, p, steps, warmup, flush):
+    """Per-step device time of the whole call and of the fused kernel (ms lists).
+    `flush` is the L2 flush buffer, or None when replicas rotate."""
     import ctypes
 
     import paged_quantized_kv_attention_b200 as pa
     stream = torch.cuda.current_stream()
-    args = (d["q"], d["k_cache"], d["v_cache"], d["k_scale"], d["v_scale"], d["block_table"],
-            d["seqlens_k"], d["cu_seqlens_q"], d["out"])
-    for _ in range(warmup):
-        flush.zero_()
-        pa.paged_attn_forward(*args, p, stream)
+    R = len(reps)
+    for i in range(max(warmup, R)):
+        if flush is not None:
+            flush.zero_()
+        pa.paged_attn_forward(*_args(reps[i % R]), p, stream)
     torch.cuda.synchronize()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
     for e in ev:  # create the events before handing their handles to the library
@@ -195,12 +230,13 @@ def time_device(w, d, p, steps, warmup, flush):
     torch.cuda.synchronize()
     holders = []
     for i in range(steps):
-        flush.zero_()  # L2 flush, between the timed spans
+        if flush is not None:
+            flush.zero_()  # L2 flush, between the timed spans
         torch.cuda._sleep(SPIN_CYCLES)  # keep the GPU busy while the host enqueues the span
         h = _event_handles(ev[i][:2])
         holders.append(h)
         p.profile_events = ctypes.cast(h, ctypes.c_void_p)
-        pa.paged_attn_forward(*args, p, stream)
+        pa.paged_attn_forward(*_args(reps[i % R]), p, stream)
         ev[i][2].record(stream)
     torch.cuda.synchronize()
     p.profile_events = None
@@ -209,37 +245,39 @@ def time_device(w, d, p, steps, warmup, flush):
     return call_ms, kern_ms
 
 
-def time_e2e(w, d, p, steps, warmup, flush):
+def time_e2e(w, reps, p, steps, warmup, flush):
     """Through the public API with host buffers: H2D of the step's inputs from pinned
     memory, host planning, forward, D2H of the output; device-timed per step."""
     import paged_quantized_kv_attention_b200 as pa
     stream = torch.cuda.current_stream()
-    host = {k: d[k].cpu().pin_memory() for k in ("q", "block_table", "seqlens_k", "cu_seqlens_q")}
+    d0 = reps[0]
+    host = {k: d0[k].cpu().pin_memory() for k in ("q", "block_table", "seqlens_k", "cu_seqlens_q")}
     cu_h, sk_h = w["cu_seqlens_q"].copy(), w["seqlens_k"].copy()
-    out_h = torch.empty(d["out"].shape, dtype=d["out"].dtype).pin_memory()
+    out_h = torch.empty(d0["out"].shape, dtype=d0["out"].dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = out_h.numel() * out_h.element_size()
+    R = len(reps)
 
-    def one():
+    def one(d):
         for k, t in host.items():
             d[k].copy_(t, non_blocking=True)
         pa.paged_attn_plan(cu_h, sk_h, p)
-        pa.paged_attn_forward(d["q"], d["k_cache"], d["v_cache"], d["k_scale"], d["v_scale"],
-                              d["block_table"], d["seqlens_k"], d["cu_seqlens_q"], d["out"], p,
-                              stream)
+        pa.paged_attn_forward(*_args(d), p, stream)
         out_h.copy_(d["out"], non_blocking=True)
 
-    for _ in range(warmup):
-        flush.zero_()
-        one()
+    for i in range(max(warmup, R)):
+        if flush is not None:
+            flush.zero_()
+        one(reps[i % R])
     torch.cuda.synchronize()
     ms = []
-    for _ in range(steps):
-        flush.zero_()
+    for i in range(steps):
+        if flush is not None:
+            flush.zero_()
         torch.cuda._sleep(SPIN_CYCLES)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        one()
+        one(reps[i % R])
         e1.record(stream)
         e1.synchronize()
         ms.append(e0.elapsed_time(e1))
@@ -280,24 +318,26 @@ def sub_problem(w: dict, b: int) -> dict:
     return s
 
 
-def measure(name: str, steps: int, warmup: int, dev: str, flush, with_e2e: bool):
+def measure(name: str, steps: int, warmup: int, dev: str, flush_buf, with_e2e: bool):
     w = workloads.make(name)
     ab = algorithmic_bytes(w)
-    d, p = setup(w, dev)
-    call_ms, kern_ms = time_device(w, d, p, steps, warmup, flush)
+    replicas, use_flush = l2_plan(w)
+    flush = flush_buf if use_flush else None
+    reps, p = setup(w, dev, replicas)
+    call_ms, kern_ms = time_device(w, reps, p, steps, warmup, flush)
     call = statistics.mean(call_ms)
     kern = statistics.mean(kern_ms)
     peak, peak_kind = measured_peaks()
     res = dict(w=w, ab=ab, p=p, call_ms=call, kern_ms=kern,
                value=ab["total"] / (call * 1e-3) / 1e9,
                kernel_gbs=ab["fwd"] / (kern * 1e-3) / 1e9, peak=peak, peak_kind=peak_kind,
-               launches_per_step=1)
+               launches_per_step=1, l2=l2_desc(replicas, use_flush, w))
     if with_e2e:
-        e2e_ms, h2d, d2h = time_e2e(w, d, p, max(5, steps // 2), 2, flush)
+        e2e_ms, h2d, d2h = time_e2e(w, reps, p, max(5, steps // 2), 2, flush)
         res["e2e"] = dict(value=ab["total"] / (statistics.mean(e2e_ms) * 1e-3) / 1e9,
                           unit="GB/s", h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
                           ms_per_step=statistics.mean(e2e_ms))
-    del d
+    del reps
     torch.cuda.empty_cache()
     return res
 
@@ -309,7 +349,7 @@ def summary_of(name, r):
             "kernel_us": round(r["kern_ms"] * 1e3, 2),
             "kernel_gbs": round(r["kernel_gbs"], 1),
             "kernel_frac_of_%s_peak" % r["peak_kind"]: round(r["kernel_gbs"] / r["peak"], 3),
-            "num_splits": r["p"].num_splits, "algorithmic_bytes": r["ab"]["total"]}
+            "num_splits": r["p"].num_splits, "algorithmic_bytes": r["ab"]["total"], "l2": r["l2"]}
 
 
 def run_ours(args):
@@ -376,7 +416,7 @@ def run_ours(args):
                    "kv_dtype": workloads.KV_NAMES[r["w"]["kv_dtype"]],
                    "global_batch": r["w"]["batch"] * world, "seq_len": int(r["w"]["seqlens_k"].max()),
                    "parallelism": "replicas x%d" % world,
-                   "l2": "flushed between steps (256 MB write), per-step CUDA events",
+                   "l2": r["l2"], "timing": "per-step CUDA events on the launching stream",
                    "num_splits": r["p"].num_splits, "blocks_per_split": r["p"].blocks_per_split},
         "us_per_call": round(r["call_ms"] * 1e3, 3),
         "tokens_per_s": round(world * ab["tokens"] / (r["call_ms"] * 1e-3), 1),

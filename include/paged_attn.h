@@ -112,19 +112,20 @@ typedef struct {
   float softmax_scale;    /* 0 -> 1/sqrt(head_size) */
   int causal;             /* 1: bottom-right causal mask for new tokens; 0: none */
   int num_sms;            /* 0 -> SM count of the current device (148 if none) */
-  int split_blocks;       /* 0: planner decides; > 0: force this many KV blocks per
-                             split; < 0: never split */
+  int split_blocks;       /* 0: planner decides; > 0: use this split target T (KV
+                             blocks per split); < 0: never split */
   /* ---- filled by paged_attn_plan ---- */
   int total_q;            /* cu_seqlens_q[batch] */
   int max_query_len;      /* exact max_b (cu[b+1] - cu[b]) */
   int max_seqlen_k;       /* max_b seqlens_k[b] */
-  int rows_per_cta;       /* query rows (tokens x group heads) per CTA: 4, 8 or 16
-                             (4: at most 4 rows per sequence and KV head, the fp16
-                             residual of the folded query rides in the idle MMA
-                             columns) */
+  int rows_per_cta;       /* query rows (tokens x group heads) per work item: 4, 8
+                             or 16 (4: at most 4 rows per sequence and KV head) */
   int num_row_groups;     /* ceil(max_query_len * H/Hk / rows_per_cta) */
-  int num_splits;         /* KV splits of the longest sequence (1 = no split) */
-  int blocks_per_split;   /* KV blocks per split */
+  int num_splits;         /* most KV splits of any sequence (1 = no split); the
+                             workspace holds this many partials per row */
+  int blocks_per_split;   /* split target T in KV blocks: a sequence with n blocks
+                             is cut into min(num_splits, ceil(n / T)) equal splits */
+  int num_work_items;     /* work items (sequence, KV head, row group, split) */
   size_t workspace_bytes; /* bytes the forward call needs (>= 256) */
   /* ---- supplied by the caller before paged_attn_forward ---- */
   void* workspace;        /* device memory, 256-byte aligned, >= workspace_bytes,
@@ -142,8 +143,9 @@ typedef struct {
 /* Host-side planner.  Validates the problem, computes the exact max_query_len
  * and max_seqlen_k from HOST copies of cu_seqlens_q [batch+1] and seqlens_k
  * [batch] (the exact-max_query_len page, Code analysis 1), chooses the KV split
- * (split-KV when B*Hk*row groups underfills the SMs and there is more than one
- * block per sequence, after the GQA GEMV decode page's flash-decoding rule), and
+ * (flash decoding after the GQA GEMV decode page's rule: the split target that
+ * makes the work items fill the device's resident CTA slots in the least
+ * estimated time; no split when the units alone do), and
  * reports the workspace size.  Launches nothing; needs no GPU.  Contract checks:
  * cu[0] == 0, 0 <= q_b <= seqlens_k[b] <= max_blocks_per_seq * block_size. */
 pa_status paged_attn_plan(const int32_t* cu_seqlens_q_host, const int32_t* seqlens_k_host,

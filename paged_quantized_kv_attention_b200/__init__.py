@@ -47,7 +47,8 @@ class paged_attn_params(ctypes.Structure):  # noqa: N801 (mirrors the C struct n
                 ("total_q", ctypes.c_int), ("max_query_len", ctypes.c_int),
                 ("max_seqlen_k", ctypes.c_int), ("rows_per_cta", ctypes.c_int),
                 ("num_row_groups", ctypes.c_int), ("num_splits", ctypes.c_int),
-                ("blocks_per_split", ctypes.c_int), ("workspace_bytes", ctypes.c_size_t),
+                ("blocks_per_split", ctypes.c_int), ("num_work_items", ctypes.c_int),
+                ("workspace_bytes", ctypes.c_size_t),
                 ("workspace", ctypes.c_void_p), ("profile_events", ctypes.c_void_p)]
 
 

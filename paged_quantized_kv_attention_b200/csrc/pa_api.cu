@@ -41,10 +41,8 @@ pa_status ok() {
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 constexpr size_t kHeaderBytes = pa::kWsHeaderBytes;  // error word + reserved
-constexpr int kCtasPerSm = 3;          // typical resident forward CTAs per SM
-constexpr int kItemsPerCta = 4;        // work items per resident CTA wanted for balance
-constexpr int64_t kMinSplitBytes = 64 << 10;  // smallest KV split worth a partial write
 constexpr int kMaxSplits = 128;        // merge weights of one row group fit in shared memory
+constexpr double kItemCostBytes = 16384.0;  // fixed cost of one work item, in KV bytes
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -211,33 +209,78 @@ pa_status paged_attn_plan(const int32_t* cu_seqlens_q_host, const int32_t* seqle
   p->max_query_len = max_q;
   p->max_seqlen_k = max_k;
   const int64_t max_rows = static_cast<int64_t>(max_q) * G;
-  // 4 rows: decode with G <= 4, fp16 residuals packed into the idle MMA columns
+  // 4 rows: at most 4 rows per (sequence, KV head) (a decode step with G <= 4)
   p->rows_per_cta = max_rows > 8 ? 16 : (max_rows > 4 ? 8 : 4);
   p->num_row_groups = static_cast<int>((max_rows + p->rows_per_cta - 1) / p->rows_per_cta);
   const int sms = p->num_sms > 0 ? p->num_sms : current_sm_count();
   const int max_nblk = (max_k + bs - 1) / bs;
-  int bps = max_nblk > 0 ? max_nblk : 1;
+  // Split target T (KV blocks per split).  Automatic choice: the T that minimises
+  // an estimate of the makespan of the work items over the resident CTAs:
+  // (rounds - 1) * mean item + largest item + rounds * per-item cost + the split
+  // partials' write and read spread over the CTAs + the final merge (latency
+  // and one CTA reading the partials) when anything is split (flash decoding after the
+  // GQA GEMV decode page, Code analysis 2, sized for the resident CTA slots).
+  const int rows = p->rows_per_cta;
+  const int Hk = p->kv_num_heads;
+  const double block_bytes = 2.0 * bs * cache_row_bytes(p->kv_dtype, p->head_size);
+  const double item_cost = kItemCostBytes / block_bytes;
+  const double part_cost = 2.0 * rows * p->head_size * 4.0 / block_bytes;
+  const int64_t slots = static_cast<int64_t>(sms) *
+                        pa::forward_ctas_per_sm(p->kv_dtype, p->head_size, bs, rows);
+  auto count = [&](int T, int64_t* items, int64_t* split_items, int* max_bps, int* max_ns,
+                   double* work) {
+    *items = *split_items = 0;
+    *max_bps = *max_ns = 0;
+    *work = 0.0;
+    for (int b = 0; b < B; ++b) {
+      const int qb = cu_seqlens_q_host[b + 1] - cu_seqlens_q_host[b];
+      if (qb == 0) continue;
+      const int64_t units = static_cast<int64_t>(Hk) * ((static_cast<int64_t>(qb) * G + rows - 1) / rows);
+      const int nblk = (seqlens_k_host[b] + bs - 1) / bs;
+      int ns, bps;
+      pa::split_geometry(nblk, T, kMaxSplits, &ns, &bps);
+      *items += units * ns;
+      if (ns > 1) *split_items += units * ns;
+      if (bps > *max_bps) *max_bps = bps;
+      if (ns > *max_ns) *max_ns = ns;
+      *work += static_cast<double>(units) * nblk;
+    }
+  };
+  int T = max_nblk > 0 ? max_nblk : 1;
   if (p->split_blocks > 0) {
-    bps = p->split_blocks;
-  } else if (p->split_blocks == 0) {
-    // Split the KV of a unit (flash decoding) when the units alone would leave
-    // the persistent CTAs with fewer than kItemsPerCta items each; splits carry
-    // at least kMinSplitBytes of K+V so the partial write stays small.
-    const int64_t units = static_cast<int64_t>(B) * p->kv_num_heads * p->num_row_groups;
-    const int64_t want_items = static_cast<int64_t>(sms) * kCtasPerSm * kItemsPerCta;
-    const int64_t block_bytes = 2LL * bs * cache_row_bytes(p->kv_dtype, p->head_size);
-    const int64_t min_bps = (kMinSplitBytes + block_bytes - 1) / block_bytes;
-    if (units > 0 && units < want_items && max_nblk > min_bps) {
-      const int64_t work = total_blocks * p->kv_num_heads * p->num_row_groups;
-      int64_t b2 = (work + want_items - 1) / want_items;
-      if (b2 < min_bps) b2 = min_bps;
-      bps = static_cast<int>(b2);
+    T = p->split_blocks;
+  } else if (p->split_blocks == 0 && max_nblk > 1 && total_q > 0) {
+    double best = -1.0;
+    int prev_T = -1;
+    for (int sp = 1; sp <= kMaxSplits && sp <= max_nblk; sp += (sp < 16 ? 1 : sp / 8)) {
+      const int Tc = (max_nblk + sp - 1) / sp;
+      if (Tc == prev_T) continue;
+      prev_T = Tc;
+      int64_t items, split_items;
+      int max_bps, max_ns;
+      double work;
+      count(Tc, &items, &split_items, &max_bps, &max_ns, &work);
+      if (items <= 0) break;
+      const int64_t rounds = (items + slots - 1) / slots;
+      // a split adds the last arrival's merge: its latency and its read of all
+      // the unit's partials by one CTA
+      const double est = (rounds - 1) * (work / items) + max_bps + rounds * item_cost +
+                         split_items * part_cost / slots +
+                         (max_ns > 1 ? 2.0 * item_cost + 0.5 * max_ns * part_cost : 0.0);
+      if (best < 0.0 || est < best) {
+        best = est;
+        T = Tc;
+      }
     }
   }
-  if (bps > max_nblk) bps = max_nblk > 0 ? max_nblk : 1;
-  if (max_nblk > 0 && (max_nblk + bps - 1) / bps > kMaxSplits) bps = (max_nblk + kMaxSplits - 1) / kMaxSplits;
-  p->blocks_per_split = bps;
-  p->num_splits = max_nblk > 0 ? (max_nblk + bps - 1) / bps : 1;
+  int64_t items = 0, split_items = 0;
+  int max_bps = 0, max_ns = 1;
+  double work = 0.0;
+  count(T, &items, &split_items, &max_bps, &max_ns, &work);
+  if (items >= (int64_t(1) << 31)) return fail(PA_ERR_UNSUPPORTED, "too many work items");
+  p->blocks_per_split = T;
+  p->num_splits = max_ns > 0 ? max_ns : 1;
+  p->num_work_items = static_cast<int>(items);
   const size_t ws = ws_layout(p).total;
   p->workspace_bytes = ws;
   if (workspace_bytes_needed) *workspace_bytes_needed = ws;
@@ -263,11 +306,9 @@ pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_c
   const int G = p->num_heads / p->kv_num_heads;
   const int64_t need_rg = (static_cast<int64_t>(p->max_query_len) * G + p->rows_per_cta - 1) /
                           p->rows_per_cta;
-  if (p->num_row_groups != need_rg || p->num_splits < 1 || p->blocks_per_split < 1)
+  if (p->num_row_groups != need_rg || p->num_splits < 1 || p->blocks_per_split < 1 ||
+      p->num_work_items < 0)
     return fail(PA_ERR_INVALID_ARG, "params were not filled by paged_attn_plan (grid)");
-  if (static_cast<int64_t>(p->num_splits) * p->blocks_per_split <
-      (static_cast<int64_t>(p->max_seqlen_k) + p->block_size - 1) / p->block_size)
-    return fail(PA_ERR_INVALID_ARG, "num_splits * blocks_per_split does not cover max_seqlen_k");
   if (!q || !k_cache || !v_cache || !k_scale || !v_scale || !block_table || !seqlens_k ||
       !cu_seqlens_q || !out)
     return fail(PA_ERR_INVALID_ARG, "a device pointer argument is NULL");
@@ -315,12 +356,9 @@ pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_c
   a.out_bf16 = p->out_dtype == PA_BF16;
   a.causal = p->causal;
   a.num_row_groups = p->num_row_groups;
-  a.num_splits = p->num_splits;
-  a.blocks_per_split = p->blocks_per_split;
-  const int64_t items = static_cast<int64_t>(p->batch) * p->kv_num_heads * p->num_row_groups *
-                        p->num_splits;
-  if (items >= (int64_t(1) << 31)) return fail(PA_ERR_UNSUPPORTED, "too many work items");
-  a.num_items = static_cast<int>(items);
+  a.max_splits = p->num_splits;
+  a.split_target = p->blocks_per_split;
+  a.num_items = p->num_work_items;
   a.num_sms = p->num_sms > 0 ? p->num_sms : current_sm_count();
   const float scale = p->softmax_scale > 0.f ? p->softmax_scale
                                              : 1.0f / sqrtf(static_cast<float>(p->head_size));

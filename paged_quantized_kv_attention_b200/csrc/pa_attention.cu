@@ -1,35 +1,45 @@
 // pa_attention.cu -- fused paged quantised-KV GQA attention for sm_100a.
 //
-// Work items.  A unit is one (sequence, KV head, group of query rows); its rows
-// are (new token, query head of the group) pairs that read the same keys, so the
-// GQA group x new tokens form the N side of a tensor-core tile, keys the M side
-// ("swap-AB"), channels the K side.  A unit's key blocks may be split into
-// several items (flash decoding).  The kernel is persistent: one CTA per
-// resident slot, items handed out by an atomic counter in the workspace.
+// Work items.  A unit is one (sequence, KV head, group of query rows): the rows
+// are the (new token, query head of the GQA group) pairs that read the same
+// keys.  They are the N side of the tensor-core tiles, keys the M side
+// ("swap-AB"), channels the K side.  A sequence with n KV blocks is split into
+// ceil(n / T) items of equal size (flash decoding), T chosen by the planner so
+// that the items fill the resident CTAs in whole rounds.  Items are numbered
+// densely over the sequences with new tokens: the producer warp of every CTA
+// computes the per-sequence item counts and their prefix sums once, from the
+// device lengths.  The kernel is persistent: CTA i starts with item i and then
+// pulls items from an atomic counter in the workspace.
 //
-// Per CTA:
-//   producer warp : fetches the next item, loads its lengths, bulk-copies its
-//                   query rows and both per-channel scale rows into one of two
-//                   item slots, then streams its KV blocks (block_table -> two
-//                   3-D TMA boxes per block, K rows and V rows of one head) into
-//                   a swizzled ring of stages, straight after the previous
-//                   item's blocks, so the next item's data lands while the
-//                   consumers finish the current one.
-//   consumer warps: per item: fold the K scale into the queries, then per 32
-//                   keys: ldmatrix (K) -> QK MMA (INT8/INT4 codes straight into
-//                   mma.sync m16n8k32 s8/u8 x s8 against four int8 digits of the
-//                   folded query, exact int32 accumulation; FP8 codes converted
-//                   to fp16 in registers for m16n8k16 against an fp16 high part
-//                   plus residual) -> online softmax in the exp2 domain whose
-//                   running maximum is only raised (shuffle reduction and
-//                   rescale) when a logit exceeds it by more than 2^8 -> P^T to
-//                   fp16 with movmatrix -> ldmatrix.trans (V) -> exact
-//                   code->fp16 in registers -> mma.sync m16n8k16 into O^T.
-// The four consumer warps take alternate 32-key groups and merge (m, l, O)
-// through shared memory at the end of an item, where the per-channel V scale is
-// applied once.  A split item writes a normalised partial and its log2-sum-exp;
-// the last item of a unit to finish (arrival counter in the workspace) merges
-// them and resets the counter.
+// Per CTA, one producer warp and four consumer warps:
+//   producer : per item, bulk-copies the query rows and both per-channel scale
+//              rows into one of two item slots, then streams the item's KV
+//              blocks (block table -> two 3-D TMA boxes per block: the K rows and
+//              the V rows of one head) into the consumers' stage rings, straight
+//              after the previous item's blocks.  The next item's index and block
+//              table entries are fetched while the current ones stream.
+//   consumers: per item, the four warps fold the K scale into the queries and
+//              encode them as B-operand fragments in shared memory (each warp a
+//              quarter of the work); then each warp takes alternate 32-key groups:
+//              ldmatrix (K) -> QK on the tensor cores -> online softmax (exp2
+//              domain, running maximum raised only when a logit exceeds it by more
+//              than 2^8) -> P^T in fp16 -> ldmatrix.trans (V) -> code -> fp16 ->
+//              PV MMA; finally the warps' (m, l, O) are merged through shared
+//              memory, the V scale applied once, and the result (or a split
+//              partial and its log2-sum-exp) stored.  The last split of a unit to
+//              finish merges the partials (arrival counter in the workspace).
+//
+// QK arithmetic.  INT8 and INT4 caches: the folded query q'' = q' 2^(6 - e_q)
+// (|q''| < 64) is split into signed int8 digits q'' = d0 + d1 2^-7 + d2 2^-14
+// (+ d3 2^-21), each the B operand of an exact mma.sync m16n8k32 s8 x s8 -> s32
+// whose A operand is the raw cache byte (INT4: the nibble shifted into the high
+// half of a byte, 16 x code).  FP8 caches: codes -> fp16 in registers, q' as an
+// fp16 high part plus an fp16 residual.  With at most 4 rows per item, MMA column
+// n carries row n / 2, so a thread holds every digit (or both parts) of one row.
+// PV arithmetic.  V codes -> fp16 exactly with one byte permute (INT8:
+// 1152 + code) or one logic op (INT4: 1032 + code, 1152 + 16 code); the constant
+// is removed once at the end using the row sum of P, which a ones-matrix MMA
+// accumulates from exactly the fp16 P values the PV MMA consumed.
 //
 // Sources: the per-channel K scale folded into Q with a power-of-two normaliser
 // (INT4 paged-KV page, onnxruntime PR 32515, Code analysis 3); INT8 codes kept
@@ -37,8 +47,8 @@
 // accumulation (INT8-KV tensor-core page, onnxruntime PR 33707, Code analysis
 // 1); online softmax, masking and the flash-decoding split with a partials
 // buffer (GQA GEMV decode page, onnxruntime PR 29216, Code analysis 1-2); the
-// grid of units sized by the exact max_query_len (exact max_query_len page,
-// onnxruntime PR 28409, Code analysis 2).
+// units sized by the exact max_query_len (exact max_query_len page, onnxruntime
+// PR 28409, Code analysis 2).
 #include <math.h>
 
 #include <atomic>
@@ -48,12 +58,16 @@
 
 namespace pa {
 
-// NT: 8-row n-tiles per CTA (rows = 8 NT).  LOPACK (NT = 1 only): the unit has at
-// most 4 rows; B-operand columns 0..3 carry one half of each pair of query parts
-// (fp16 high part, or int8 digits 0 and 2) and columns 4..7 the other (residual,
-// or digits 1 and 3), halving the QK MMAs.
-template <int KV, int D, int BS, int NT, bool LOPACK>
+constexpr uint32_t kFull = 0xffffffffu;
+constexpr uint32_t kOnesH2 = 0x3C003C00u;  // fp16x2 (1, 1)
+
+// NT: 8-column n-tiles per item (rows = 8 NT).  LP: at most 4 rows per item;
+// MMA column n carries row n / 2 (QK: the two halves of a digit/part pair;
+// PV: the row twice).
+template <int KV, int D, int BS, int NT, bool LP>
 struct Cfg {
+  static_assert(!LP || NT == 1, "row-pair packing uses one n-tile");
+  static constexpr bool kInt = (KV != PA_KV_FP8_E4M3);
   static constexpr int kCHS = (KV == PA_KV_INT4) ? D / 2 : D;  // cache bytes per row
   static constexpr int kTile = BS * kCHS;                       // one block, one head
   static constexpr int kStageBytes = 2 * kTile;                 // K + V
@@ -70,37 +84,47 @@ struct Cfg {
   static constexpr int kSWRaw = 65536 / (kWarps * kStageBytes);
   static constexpr int kSW = kSWRaw < 2 * kBPI ? 2 * kBPI : (kSWRaw > 16 ? 16 : kSWRaw);
   static constexpr int kStages = kWarps * kSW;
-  // producer group: whole warp iterations, at most kSW blocks per warp, <= 32 lanes
+  // producer group: whole warp iterations, at most kSW blocks of any warp, <= 32 lanes
   static constexpr int kItPerGroupRaw = (kSW < 8 ? kSW : 8) / kBPI;
   static constexpr int kGroup = kWarps * kBPI * (kItPerGroupRaw < 1 ? 1 : kItPerGroupRaw);
-  static constexpr int kRows = 8 * NT;
-  static constexpr bool kImma = (KV != PA_KV_FP8_E4M3);         // QK on int8 tensor cores
-  static constexpr int kAcc = LOPACK ? 2 : 4;                   // int32 QK accumulators
-  static constexpr int kQRegs = kImma ? (D / 32) * kAcc * 2 : (D / 16) * (LOPACK ? 2 : 4);
-  static constexpr int kQElems = D / 4;                         // query channels per thread
+  static constexpr int kRows = LP ? 4 : 8 * NT;
+  // QK accumulator sets per n-tile: integer digits (LP: 2 x 2 digits; else 3),
+  // FP8 parts (LP: hi|lo in one; else hi, lo)
+  static constexpr int kAcc = kInt ? (LP ? 2 : 3) : (LP ? 1 : 2);
+  static constexpr int kDigits = LP ? 4 : 3;
+  static constexpr int kKSteps = kInt ? D / 32 : D / 16;
+  static constexpr int kQWords = kKSteps * kAcc * 2;            // B-fragment words per lane
+  static constexpr int kQStride =
+      ((kQWords / 4) % 2 == 0 && kQWords < 32) ? kQWords + 4 : kQWords;  // lds.128 banks
+  static constexpr int kUnits = D / 4;                          // 4-channel prologue units per row
+  static constexpr int kSlices = LP ? 3 : 1;                    // warp-merge buffers
   static constexpr int kMaxSplits = 128;
-  // shared memory map (all offsets from the 1024-aligned base)
+  // shared memory map (offsets from the 1024-aligned base)
   static constexpr int kRingBytes = kStages * kStageBytes;
   static constexpr int kQBytes = kRows * D * 2;                 // query rows of one item slot
   static constexpr int kQOff = kRingBytes;                      // 2 slots
   static constexpr int kKsOff = kQOff + 2 * kQBytes;            // k_scale rows, 2 slots
   static constexpr int kVsOff = kKsOff + 2 * D * 4;             // v_scale rows, 2 slots
-  static constexpr int kEpiOff = kVsOff + 2 * D * 4;            // per-warp partial outputs,
-  static constexpr int kEpiBytes =                              // later the split weights
-      (D > kMaxSplits ? D : kMaxSplits) * kRows * 4;
-  static constexpr int kBarOff = kEpiOff + kEpiBytes;
+  static constexpr int kUnionOff = kVsOff + 2 * D * 4;          // fragments | merge slices | weights
+  static constexpr int kFragBytes = NT * 32 * kQStride * 4;
+  static constexpr int kSliceBytes = kRows * D * 4;
+  static constexpr int kWtsBytes = kMaxSplits * kRows * 4;
+  static constexpr int kU0 = kFragBytes > kSlices * kSliceBytes ? kFragBytes : kSlices * kSliceBytes;
+  static constexpr int kUnionBytes = kU0 > kWtsBytes ? kU0 : kWtsBytes;
+  static constexpr int kBarOff = kUnionOff + kUnionBytes;
   static constexpr int kNumBars = 2 * kStages + 4;              // full, empty, item full/empty
   static constexpr int kDescOff = kBarOff + kNumBars * 8;
-  static constexpr int kStatOff = kDescOff + 2 * 64;
-  static constexpr int kFlagOff = kStatOff + 2 * kWarps * kRows * 4;
+  static constexpr int kMLOff = kDescOff + 2 * 64;              // merge m, l: [kSlices][2][kRows]
+  static constexpr int kCOff = kMLOff + kSlices * 2 * kRows * 4;  // row logit multipliers
+  static constexpr int kFlagOff = kCOff + kRows * 4;
   static constexpr int kSmemBytes = kFlagOff + 16;
   static_assert(kChunks % 2 == 0, "ldmatrix.x4 covers two 16-byte chunks");
   static_assert(kTile % ((kSwzMask + 1) * 128) == 0, "tiles keep the swizzle-atom alignment");
-  static_assert(!LOPACK || NT == 1, "residual packing needs a single n-tile");
   static_assert(kTPI == 2, "two 16-key tiles per warp iteration");
   static_assert(kStages <= 64, "stage count");
   static_assert(kGroup <= 32 && kGroup / (kWarps * kBPI) * kBPI <= kSW, "producer group");
-  static_assert(kMaxSplits * kRows * 4 <= kEpiBytes, "split weights fit in the epilogue buffer");
+  static_assert(kQWords % 4 == 0 && kQStride % 4 == 0, "fragment rows are lds.128 aligned");
+  static_assert(kUnionOff % 16 == 0, "fragment area alignment");
 };
 
 // One work item as published by the producer to the consumers (64 bytes).
@@ -127,30 +151,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
 
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-// Channel of the i-th query value a thread contributes to the QK B operand (the
-// thread with index tig in its quad).  It matches the channels ldmatrix hands the
-// same thread for the K operand.  Element i = 4 * word + byte (integer caches:
-// word = 2 s + r for k32-step s and B register r; FP8: i = 4 s + j for 16-channel
-// k-step s and half j).
-template <int KV>
-__device__ __forceinline__ int q_channel(int i, int tig) {
-  const int wd = i >> 2, e = i & 3;
-  if constexpr (KV == PA_KV_INT8) {
-    return 32 * (wd >> 1) + 16 * (wd & 1) + 4 * tig + e;
-  } else if constexpr (KV == PA_KV_INT4) {
-    return 32 * (wd >> 1) + 8 * tig + 2 * e + (wd & 1);
-  } else {
-    return 16 * wd + 4 * tig + e;
-  }
-}
-
-// First of the two adjacent output dims held by M rows g / g+8 of PV m-tile mt.
-template <int KV>
-__device__ __forceinline__ int out_dim(int mt, int g) {
-  if constexpr (KV == PA_KV_INT4) return 32 * (mt >> 1) + 4 * g + 2 * (mt & 1);
-  return 16 * mt + 2 * g;
-}
-
 // One bulk copy (global -> shared) completing on an mbarrier.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
                                           uint32_t bar) {
@@ -161,27 +161,52 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
-// Rows, keys and block range of work item w, from the device lengths of its
-// sequence.  Returns false (and leaves d.valid = 0) when the item has no work:
-// no new tokens, fewer rows than its row group, or a split past the last block.
+// First of the two adjacent output dims held by accumulator elements c0 / c2 of
+// PV m-tile mt for a thread with group index g.
+template <int KV>
+__device__ __forceinline__ int out_dim(int mt, int g) {
+  if constexpr (KV == PA_KV_INT4) return 32 * (mt >> 1) + 4 * g + 2 * (mt & 1);
+  return 16 * mt + 2 * g;
+}
+
+// Column offset of dim pair d in a merge slice row (spreads the four row groups
+// of a warp over the banks).
+__device__ __forceinline__ int slice_col(int d, int sw) { return d ^ (sw << 3); }
+
+// Items of sequence b (0 if it has no new tokens or its lengths are invalid).
 template <int BS>
-__device__ __forceinline__ bool decode_item(const FwdArgs& a, int rows_cta, int w, int q0,
-                                            int q1, int Lb, ItemDesc& d) {
-  const int u = w / a.num_splits;
-  d.valid = 0;
-  d.split = w % a.num_splits;
-  d.rg = u % a.num_row_groups;
-  d.kv = (u / a.num_row_groups) % a.Hk;
-  d.b = u / (a.num_row_groups * a.Hk);
-  const int qb = q1 - q0;
-  if (q0 < 0 || qb < 0 || qb > Lb || q0 + qb > a.total_q ||
-      static_cast<long long>(Lb) > static_cast<long long>(a.maxb) * BS) {
-    record_error(a.err, PA_DEVERR_BAD_LENGTH);
-    return false;
+__device__ __forceinline__ int seq_items(const FwdArgs& a, int rows_cta, int q0, int qb, int Lb,
+                                         bool& bad) {
+  bad = (q0 < 0 || qb < 0 || qb > Lb || q0 + qb > a.total_q ||
+         static_cast<long long>(Lb) > static_cast<long long>(a.maxb) * BS);
+  if (bad || qb == 0) return 0;
+  const int rg = (qb * a.G + rows_cta - 1) / rows_cta;
+  if (rg > a.num_row_groups) {
+    bad = true;
+    return 0;
   }
-  const int R = qb * a.G;  // rows of (b, kv): row r = token (r / G), head kv*G + r % G
+  int ns, bps;
+  split_geometry((Lb + BS - 1) / BS, a.split_target, a.max_splits, &ns, &bps);
+  return a.Hk * rg * ns;
+}
+
+// Rows, keys and block range of item `local` of sequence b.  Returns false (and
+// leaves d.valid = 0) when the item has no keys (a causal row group that ends
+// before this split starts).
+template <int BS>
+__device__ __forceinline__ bool decode_item(const FwdArgs& a, int rows_cta, int b, int local,
+                                            int q0, int qb, int Lb, ItemDesc& d) {
+  d.valid = 0;
+  const int R = qb * a.G;  // rows of (b, kv): row r = token r / G, head kv * G + r % G
+  const int rg_n = (R + rows_cta - 1) / rows_cta;
+  int ns, bps;
+  split_geometry((Lb + BS - 1) / BS, a.split_target, a.max_splits, &ns, &bps);
+  d.split = local % ns;
+  const int rest = local / ns;
+  d.rg = rest % rg_n;
+  d.kv = rest / rg_n;
+  d.b = b;
   d.row0 = d.rg * rows_cta;
-  if (d.row0 >= R) return false;
   d.row_end = min(R, d.row0 + rows_cta);
   d.q0 = q0;
   d.Lb = Lb;
@@ -190,10 +215,10 @@ __device__ __forceinline__ bool decode_item(const FwdArgs& a, int rows_cta, int 
   d.kmax = a.causal ? d.past + i_last + 1 : Lb;    // keys seen by some row
   d.kfull = a.causal ? d.past + i_first + 1 : Lb;  // keys seen by every row
   const int nblk = (d.kmax + BS - 1) / BS;
-  d.nsplit = (nblk + a.blocks_per_split - 1) / a.blocks_per_split;
-  if (d.split >= d.nsplit) return false;
-  d.blk_begin = d.split * a.blocks_per_split;
-  d.nloc = min(nblk, d.blk_begin + a.blocks_per_split) - d.blk_begin;
+  d.nsplit = (nblk + bps - 1) / bps;               // splits of this unit that have keys
+  d.blk_begin = d.split * bps;
+  if (d.blk_begin >= nblk) return false;
+  d.nloc = min(nblk, d.blk_begin + bps) - d.blk_begin;
   d.valid = 1;
   return true;
 }
@@ -207,11 +232,129 @@ __device__ __forceinline__ int warp_blocks(int nloc, int w) {
   return full * BPI + (rem <= 0 ? 0 : (rem < BPI ? rem : BPI));
 }
 
-template <int KV, int D, int BS, int NT, bool LOPACK>
-__global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LOPACK>::kThreads)
+// ---------------------------------------------------------------------------
+// Query fragments.  The 128 consumer threads fold k_scale into the item's query
+// rows and write every lane's B-operand words to `frag` (lane-major, kQStride
+// words per lane), plus each row's logit multiplier C to `rowc`:
+//   integer caches: logit (log2 units) = C 2^-6 sum_d code_d q''_d, q'' digits
+//   FP8           : logit = C sum_d code_d (hi_d + lo_d)
+// with C = softmax_scale log2(e) 2^(e_kv + e_q).
+// Word layout (per n-tile, per lane (g, tig)): word (s * kAcc + i) * 2 + r is
+// b-register r of k-step s for accumulator set i.  Channel of byte / half e:
+//   INT8: 32 s + 16 r + 4 tig + e     INT4: 32 s + 8 tig + 2 e + r
+//   FP8 : 16 s + 4 tig + 2 r + e (e < 2, one fp16 per half)
+// These match the channels ldmatrix hands the same thread for the K operand.
+template <int KV, int D, int BS, int NT, bool LP>
+__device__ __forceinline__ void build_fragments(const FwdArgs& a, const uint8_t* sq,
+                                                const float* sks, int nrows, uint32_t* frag,
+                                                float* rowc, int tid) {
+  using C = Cfg<KV, D, BS, NT, LP>;
+  const int lane = tid & 31;
+  float ksmax = 0.f;
+#pragma unroll
+  for (int d = lane; d < D; d += 32) ksmax = fmaxf(ksmax, fabsf(sks[d]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ksmax = fmaxf(ksmax, __shfl_xor_sync(kFull, ksmax, o));
+  if (!isfinite(ksmax) && tid == 0) record_error(a.err, PA_DEVERR_BAD_SCALE);
+  int e_kv = 0;
+  (void)frexpf(ksmax, &e_kv);
+  const float f_kv = ldexpf(1.f, -e_kv);
+  const __half* q16 = reinterpret_cast<const __half*>(sq);
+  const __nv_bfloat16* qbf = reinterpret_cast<const __nv_bfloat16*>(sq);
+  constexpr int kU = C::kUnits;  // 32 (D = 128) or 16 lanes per row
+  for (int idx = tid; idx < C::kRows * kU; idx += 128) {
+    const int row = idx / kU, u = idx % kU;
+    const bool valid = row < nrows;
+    int s, r, tq, ch0, cstep;
+    if constexpr (KV == PA_KV_INT8) {
+      s = u >> 3; r = (u >> 2) & 1; tq = u & 3; ch0 = 32 * s + 16 * r + 4 * tq; cstep = 1;
+    } else if constexpr (KV == PA_KV_INT4) {
+      s = u >> 3; r = (u >> 2) & 1; tq = u & 3; ch0 = 32 * s + 8 * tq + r; cstep = 2;
+    } else {
+      s = u >> 2; r = 0; tq = u & 3; ch0 = 16 * s + 4 * tq; cstep = 1;
+    }
+    float w[4];
+    float rmax = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int ch = ch0 + e * cstep;
+      float x = 0.f;
+      if (valid) x = a.q_bf16 ? __bfloat162float(qbf[row * D + ch]) : __half2float(q16[row * D + ch]);
+      w[e] = x * (sks[ch] * f_kv);
+      rmax = fmaxf(rmax, fabsf(w[e]));
+    }
+#pragma unroll
+    for (int o = kU / 2; o > 0; o >>= 1) rmax = fmaxf(rmax, __shfl_xor_sync(kFull, rmax, o));
+    int e_q = 0;
+    (void)frexpf(rmax, &e_q);
+    if (u == 0) rowc[row] = ldexpf(a.sm_scale_log2, e_kv + e_q);
+    const int nt = LP ? 0 : row >> 3;
+    uint32_t* fr = frag + nt * 32 * C::kQStride;
+    if constexpr (C::kInt) {
+      const float f = ldexpf(1.f, 6 - e_q);
+      uint32_t wd[C::kDigits];
+#pragma unroll
+      for (int dg = 0; dg < C::kDigits; ++dg) wd[dg] = 0u;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float v = w[e] * f;  // |v| < 64; each remainder times 128 stays within +-64
+#pragma unroll
+        for (int dg = 0; dg < C::kDigits; ++dg) {
+          const float t = rintf(v);
+          wd[dg] |= (static_cast<uint32_t>(static_cast<int>(t)) & 0xFFu) << (8 * e);
+          v = (v - t) * 128.f;
+        }
+      }
+      if constexpr (LP) {
+        // column n = 2 row + p: set i carries digit 2 i + p
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+          uint32_t* fl = fr + ((2 * row + p) * 4 + tq) * C::kQStride;
+#pragma unroll
+          for (int i = 0; i < 2; ++i) fl[(s * 2 + i) * 2 + r] = wd[2 * i + p];
+        }
+      } else {
+        uint32_t* fl = fr + ((row & 7) * 4 + tq) * C::kQStride;
+#pragma unroll
+        for (int i = 0; i < 3; ++i) fl[(s * 3 + i) * 2 + r] = wd[i];
+      }
+    } else {
+      const float f = ldexpf(1.f, -e_q);
+      float hi[4], lo[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float xn = w[e] * f;  // |xn| < 1
+        hi[e] = __half2float(__float2half_rn(xn));
+        lo[e] = xn - hi[e];
+      }
+      const uint32_t h01 = pack_f32x2_to_h2(hi[0], hi[1]), h23 = pack_f32x2_to_h2(hi[2], hi[3]);
+      const uint32_t l01 = pack_f32x2_to_h2(lo[0], lo[1]), l23 = pack_f32x2_to_h2(lo[2], lo[3]);
+      if constexpr (LP) {
+        // column n = 2 row + p: part p (0 high, 1 residual)
+        uint32_t* f0 = fr + ((2 * row) * 4 + tq) * C::kQStride;
+        uint32_t* f1 = fr + ((2 * row + 1) * 4 + tq) * C::kQStride;
+        f0[s * 2 + 0] = h01;
+        f0[s * 2 + 1] = h23;
+        f1[s * 2 + 0] = l01;
+        f1[s * 2 + 1] = l23;
+      } else {
+        uint32_t* fl = fr + ((row & 7) * 4 + tq) * C::kQStride;
+        fl[(s * 2 + 0) * 2 + 0] = h01;
+        fl[(s * 2 + 0) * 2 + 1] = h23;
+        fl[(s * 2 + 1) * 2 + 0] = l01;
+        fl[(s * 2 + 1) * 2 + 1] = l23;
+      }
+    }
+  }
+}
+
+// Registers: one n-tile fits 3 CTAs per SM (<= 136 per thread); two n-tiles
+// keep 2 CTAs per SM (<= 200 per thread).
+template <int KV, int D, int BS, int NT, bool LP>
+__global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(NT == 1 ? 128 : 200)
     pa_fwd_kernel(const __grid_constant__ CUtensorMap kmap,
                   const __grid_constant__ CUtensorMap vmap, const FwdArgs a) {
-  using C = Cfg<KV, D, BS, NT, LOPACK>;
+  using C = Cfg<KV, D, BS, NT, LP>;
   // The dynamic window starts at the CTA's shared-memory base (the kernel has no
   // static shared memory), which the 1024-byte swizzle atoms of the TMA tiles
   // need; a misaligned base is reported instead of computing garbage.
@@ -223,16 +366,17 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LOPACK>::kThreads)
   }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   ItemDesc* descs = reinterpret_cast<ItemDesc*>(smem + C::kDescOff);
-  float* sm_m = reinterpret_cast<float*>(smem + C::kStatOff);
-  float* sm_l = sm_m + C::kWarps * C::kRows;
+  float* sm_ml = reinterpret_cast<float*>(smem + C::kMLOff);
+  float* rowc = reinterpret_cast<float*>(smem + C::kCOff);
   int* sm_flag = reinterpret_cast<int*>(smem + C::kFlagOff);
-  float* epi = reinterpret_cast<float*>(smem + C::kEpiOff);
-  float* wts = epi;  // split merge weights, once the per-warp outputs are consumed
+  uint32_t* frag = reinterpret_cast<uint32_t*>(smem + C::kUnionOff);
+  float* slices = reinterpret_cast<float*>(smem + C::kUnionOff);
+  float* wts = slices;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2, tig = lane & 3;
-  const int rows_cta = LOPACK ? 4 : C::kRows;
+  constexpr int rows_cta = C::kRows;
 
   auto full_bar = [&](int s) { return smem_u32(bars + s); };
   auto empty_bar = [&](int s) { return smem_u32(bars + C::kStages + s); };
@@ -261,33 +405,144 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LOPACK>::kThreads)
       tma_prefetch_desc(&vmap);
     }
     const uint64_t policy = l2_evict_first_policy();
-    auto fetch = [&]() {
-      int w = 0;
-      if (lane == 0) w = static_cast<int>(atomicAdd(a.work, 1u));
-      return __shfl_sync(0xffffffffu, w, 0);
+    // ---- L2 prefetch of what the first items read right after the lengths:
+    // the block table, the scale rows and the queries, each CTA a slice.
+    auto prefetch_slice = [&](const void* base, size_t bytes) {
+      const size_t lines = (bytes + 127) / 128;
+      const size_t per = (lines + gridDim.x - 1) / gridDim.x;
+      const size_t lo = blockIdx.x * per;
+      const size_t hi = lo + per < lines ? lo + per : lines;
+      for (size_t l = lo + lane; l < hi; l += 32) {
+        const size_t off = l * 128 < bytes ? l * 128 : bytes - 1;
+        prefetch_l2(reinterpret_cast<const uint8_t*>(base) + off);
+      }
     };
+    prefetch_slice(a.block_table, static_cast<size_t>(a.batch) * a.maxb * 4);
+    prefetch_slice(a.k_scale, static_cast<size_t>(a.Hk) * D * 4);
+    prefetch_slice(a.v_scale, static_cast<size_t>(a.Hk) * D * 4);
+    prefetch_slice(a.q, static_cast<size_t>(a.total_q) * a.H * D * 2);
+    // ---- dense item numbering: per-sequence item counts and their prefix sums,
+    // sequence 32 k + lane in register k (up to 256 sequences); beyond that the
+    // numbering is sparse (every sequence gets the largest count; empty items
+    // are skipped).
+    constexpr int kMaxK = 8;
+    const int nk = (a.batch + 31) >> 5;
+    const bool dense = nk <= kMaxK;
+    int incl[kMaxK], cnt[kMaxK], sq0[kMaxK], sqb[kMaxK], sL[kMaxK];
+    int total = 0, per_seq = 0;
+    if (dense) {
+#pragma unroll
+      for (int k = 0; k < kMaxK; ++k) {
+        const int b = 32 * k + lane;
+        sq0[k] = sqb[k] = sL[k] = 0;
+        if (k < nk && b < a.batch) {
+          const int c0 = a.cu_seqlens_q[b], c1 = a.cu_seqlens_q[b + 1];
+          sq0[k] = c0;
+          sqb[k] = c1 - c0;
+          sL[k] = a.seqlens_k[b];
+        }
+      }
+      bool bad_any = false;
+#pragma unroll
+      for (int k = 0; k < kMaxK; ++k) {
+        incl[k] = total;
+        cnt[k] = 0;
+        if (k < nk) {  // warp-uniform
+          bool bad = false;
+          cnt[k] = (32 * k + lane < a.batch)
+                       ? seq_items<BS>(a, rows_cta, sq0[k], sqb[k], sL[k], bad)
+                       : 0;
+          bad_any |= bad;
+          int x = cnt[k];
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFull, x, o);
+            if (lane >= o) x += y;
+          }
+          incl[k] = total + x;
+          total += __shfl_sync(kFull, x, 31);
+        }
+      }
+      if (bad_any) record_error(a.err, PA_DEVERR_BAD_LENGTH);
+    } else {
+      const int max_rg = a.num_row_groups;
+      per_seq = a.Hk * max_rg * a.max_splits;
+      total = a.batch * per_seq;
+    }
+
+    // Item w -> (sequence, index within the sequence, its lengths); false when
+    // the item has no work.
+    auto locate = [&](int w, ItemDesc& d) -> bool {
+      d.valid = 0;
+      if (dense) {
+#pragma unroll
+        for (int k = 0; k < kMaxK; ++k) {
+          if (k >= nk) break;
+          const unsigned m = __ballot_sync(kFull, incl[k] > w);
+          if (m != 0u) {
+            const int l = __ffs(m) - 1;
+            const int base = __shfl_sync(kFull, incl[k] - cnt[k], l);
+            const int q0 = __shfl_sync(kFull, sq0[k], l);
+            const int qb = __shfl_sync(kFull, sqb[k], l);
+            const int Lb = __shfl_sync(kFull, sL[k], l);
+            return decode_item<BS>(a, rows_cta, 32 * k + l, w - base, q0, qb, Lb, d);
+          }
+        }
+        return false;
+      }
+      const int b = w / per_seq;
+      int v = 0;
+      if (lane == 0) v = a.cu_seqlens_q[b];
+      else if (lane == 1) v = a.cu_seqlens_q[b + 1];
+      else if (lane == 2) v = a.seqlens_k[b];
+      const int q0 = __shfl_sync(kFull, v, 0);
+      const int qb = __shfl_sync(kFull, v, 1) - q0;
+      const int Lb = __shfl_sync(kFull, v, 2);
+      bool bad = false;
+      if (seq_items<BS>(a, rows_cta, q0, qb, Lb, bad) == 0) {
+        if (bad) record_error(a.err, PA_DEVERR_BAD_LENGTH);
+        return false;
+      }
+      int local = w - b * per_seq;
+      // sparse layout: split fastest over max_splits, then row group, then head
+      const int split = local % a.max_splits;
+      const int rest = local / a.max_splits;
+      const int rg = rest % a.num_row_groups, kv = rest / a.num_row_groups;
+      const int R = qb * a.G;
+      const int rg_n = (R + rows_cta - 1) / rows_cta;
+      int ns, bps;
+      split_geometry((Lb + BS - 1) / BS, a.split_target, a.max_splits, &ns, &bps);
+      if (rg >= rg_n || split >= ns) return false;
+      return decode_item<BS>(a, rows_cta, b, (kv * rg_n + rg) * ns + split, q0, qb, Lb, d);
+    };
+
     int uses[2] = {0, 0};
     int slot = 0;
     // Blocks handed to each consumer warp so far: warp w's k-th block lives in
     // stage w * kSW + k % kSW of its own sub-ring, round k / kSW.
-    int cnt[C::kWarps] = {0, 0, 0, 0};
+    int cnt_w0 = 0, cnt_w1 = 0, cnt_w2 = 0, cnt_w3 = 0;
+    auto cnt_of = [&](int wq) {
+      return wq == 0 ? cnt_w0 : (wq == 1 ? cnt_w1 : (wq == 2 ? cnt_w2 : cnt_w3));
+    };
     bool ok = true;
-    int w = fetch();
+    int w = blockIdx.x;  // first item without an atomic
+    uint32_t w_pref = 0;
+    if (lane == 0) w_pref = atomicAdd(a.work, 1u);  // next index, in flight
+    auto next_index = [&]() {
+      const int nxt = static_cast<int>(gridDim.x + __shfl_sync(kFull, w_pref, 0));
+      if (lane == 0) w_pref = atomicAdd(a.work, 1u);
+      return nxt;
+    };
     while (ok) {
-      ItemDesc d;
-      d.valid = 0;
-      while (w < a.num_items) {
-        const int b = (w / a.num_splits) / (a.num_row_groups * a.Hk);
-        int v = 0;
-        if (lane == 0) v = a.cu_seqlens_q[b];
-        else if (lane == 1) v = a.cu_seqlens_q[b + 1];
-        else if (lane == 2) v = a.seqlens_k[b];
-        const int q0 = __shfl_sync(0xffffffffu, v, 0);
-        const int q1 = __shfl_sync(0xffffffffu, v, 1);
-        const int Lb = __shfl_sync(0xffffffffu, v, 2);
-        if (decode_item<BS>(a, rows_cta, w, q0, q1, Lb, d)) break;
-        w = fetch();
+      ItemDesc d = {};
+      while (w < total) {
+        if (locate(w, d)) break;
+        w = next_index();
       }
+      // block-table entries of the item's first group, fetched with the publish
+      const int32_t* bt = a.block_table + static_cast<size_t>(d.b) * a.maxb + d.blk_begin;
+      int phys_cur = 0;
+      if (d.valid && lane < C::kGroup && lane < d.nloc) phys_cur = __ldg(bt + lane);
       // publish the item (or the end marker) in the next slot
       if (lane == 0) {
         if (uses[slot] > 0 && !mbar_wait(item_empty(slot), (uses[slot] - 1) & 1)) {
@@ -297,9 +552,9 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LOPACK>::kThreads)
           descs[slot] = d;
           if (d.valid) {
             const uint32_t row_bytes = D * 2;
-            const uint32_t total =
+            const uint32_t tot =
                 static_cast<uint32_t>(d.row_end - d.row0) * row_bytes + 2 * D * 4;
-            mbar_arrive_expect_tx(item_full(slot), total);
+            mbar_arrive_expect_tx(item_full(slot), tot);
             const int i_first = d.row0 / a.G, i_last = (d.row_end - 1) / a.G;
             for (int i = i_first; i <= i_last; ++i) {
               const int r_lo = max(d.row0, i * a.G), r_hi = min(d.row_end, (i + 1) * a.G);
@@ -318,29 +573,29 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LOPACK>::kThreads)
           }
         }
       }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
+      ok = __shfl_sync(kFull, ok, 0);
       ++uses[slot];
       if (!ok || !d.valid) break;
-      const int w_next = fetch();  // overlaps with streaming this item
 
       // Blocks go out in groups of kGroup (whole warp iterations, at most kSW
       // blocks of any warp, so every block of a group has its own stage): lane j
-      // waits for its stage to be released, arms it and issues the two boxes,
-      // all lanes in parallel.  Item block lb belongs to warp (lb / kBPI) % 4,
-      // the same split the consumers use.
+      // waits for its stage to be released, arms it and issues the two boxes, all
+      // lanes in parallel; the next group's block-table entries are loaded first.
+      // Item block lb belongs to warp (lb / kBPI) % 4, the split the consumers use.
       constexpr int kGroup = C::kGroup;
-      const int32_t* bt = a.block_table + static_cast<size_t>(d.b) * a.maxb + d.blk_begin;
       for (int base = 0; base < d.nloc && ok; base += kGroup) {
         const int lb = base + lane;
+        int phys_nxt = 0;
+        if (lane < kGroup && lb + kGroup < d.nloc) phys_nxt = __ldg(bt + lb + kGroup);
         bool mine_ok = true;
         if (lane < kGroup && lb < d.nloc) {
-          int phys = __ldg(bt + lb);
+          int phys = phys_cur;
           if (phys < 0 || phys >= a.num_blocks) {
             record_error(a.err, PA_DEVERR_BAD_BLOCK);
             phys = a.num_blocks;  // out-of-range box: TMA fills zeros, nothing faults
           }
           const int wq = (lb / C::kBPI) % C::kWarps;
-          const int k = cnt[wq] + (lb / (C::kWarps * C::kBPI)) * C::kBPI + lb % C::kBPI;
+          const int k = cnt_of(wq) + (lb / (C::kWarps * C::kBPI)) * C::kBPI + lb % C::kBPI;
           const int s = wq * C::kSW + k % C::kSW;
           const int round = k / C::kSW;
           if (round > 0 && !mbar_wait(empty_bar(s), (round - 1) & 1)) {
@@ -351,26 +606,34 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LOPACK>::kThreads)
             tma_load_3d(smem_u32(v_tile(s)), &vmap, full_bar(s), 0, d.kv, phys * BS, policy);
           }
         }
-        ok = __all_sync(0xffffffffu, mine_ok);
+        phys_cur = phys_nxt;
+        ok = __all_sync(kFull, mine_ok);
         if (!ok && lane == 0) record_error(a.err, PA_DEVERR_TIMEOUT);
       }
-#pragma unroll
-      for (int wq = 0; wq < C::kWarps; ++wq) cnt[wq] += warp_blocks<C::kBPI>(d.nloc, wq);
+      cnt_w0 += warp_blocks<C::kBPI>(d.nloc, 0);
+      cnt_w1 += warp_blocks<C::kBPI>(d.nloc, 1);
+      cnt_w2 += warp_blocks<C::kBPI>(d.nloc, 2);
+      cnt_w3 += warp_blocks<C::kBPI>(d.nloc, 3);
       slot ^= 1;
-      w = w_next;
+      w = next_index();
     }
+    // The last prefetched index is consumed (its atomic has completed) before
+    // this CTA signs off.
+    const uint32_t last = __shfl_sync(kFull, w_pref, 0);
     // Leave no copy in flight: wait for the last box of every stage, all within
     // one bounded window (the consumers normally consumed them already).
     if (lane == 0) {
       const uint64_t deadline = global_timer_ns() + kWaitLimitNs;
       bool fine = true;
       for (int wq = 0; wq < C::kWarps; ++wq)
-        for (int j = 0; fine && j < C::kSW && j < cnt[wq]; ++j) {
-          const int last_round = (cnt[wq] - 1 - j) / C::kSW;
+        for (int j = 0; fine && j < C::kSW && j < cnt_of(wq); ++j) {
+          const int last_round = (cnt_of(wq) - 1 - j) / C::kSW;
           fine = mbar_wait_until(full_bar(wq * C::kSW + j), last_round & 1, deadline);
         }
       if (!fine) record_error(a.err, PA_DEVERR_TIMEOUT);
+      __threadfence();
       // The last CTA to finish rewinds the work counter for the next call.
+      if (last == 0xffffffffu) record_error(a.err, PA_DEVERR_BAD_LENGTH);  // (never: uses the value)
       if (atomicAdd(a.work + 1, 1u) == gridDim.x - 1) {
         a.work[0] = 0u;
         a.work[1] = 0u;
@@ -380,10 +643,17 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LOPACK>::kThreads)
   }
 
   // ======================================================== consumer warps
+  const int tid = threadIdx.x;  // 0..127
   int uses[2] = {0, 0};
   int slot = 0;
   int kc = 0;  // blocks this warp consumed so far: its k-th block is in stage
                // warp * kSW + k % kSW of its own sub-ring, round k / kSW
+  // ldmatrix lane addressing: matrix (lane >> 3) covers rows (lane & 7) + 8 * (m & 1)
+  // of a 16-row key tile and chunk (2 cp + (m >> 1)).
+  const int lm = lane >> 3;
+  const int ld_row = (lane & 7) + 8 * (lm & 1);
+  const int ld_chunk = lm >> 1;
+
   for (;;) {
     if (!mbar_wait(item_full(slot), uses[slot] & 1)) {
       if (lane == 0) record_error(a.err, PA_DEVERR_TIMEOUT);
@@ -394,185 +664,69 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LOPACK>::kThreads)
     if (!d.valid) break;
     const int kv = d.kv, rg = d.rg, b = d.b, split = d.split, q0 = d.q0;
     const int row0 = d.row0, row_end = d.row_end, past = d.past, kmax = d.kmax, kfull = d.kfull;
-    const int blk_begin = d.blk_begin, nloc = d.nloc, Lb = d.Lb, nsplit = d.nsplit;
+    const int blk_begin = d.blk_begin, nloc = d.nloc, nsplit = d.nsplit;
+    const int Lb = d.Lb;
+    const int nrows = row_end - row0;
     const float* sks = reinterpret_cast<const float*>(smem + C::kKsOff) + slot * D;
     const float* svs = reinterpret_cast<const float*>(smem + C::kVsOff) + slot * D;
     bool alive = true;
 
-    // ---- prologue: fold the K scale into the queries.  q'[d] = q[d] k_scale[d] /
-    // 2^e_kv (2^e_kv: power of two of max |k_scale| of this head), then a second
-    // power of two per row keeps |q'| < 1 for any finite input; both powers move
-    // into the per-row logit multiplier c (exp2 domain).
-    float ksmax = 0.f;
-  #pragma unroll
-    for (int d = lane; d < D; d += 32) ksmax = fmaxf(ksmax, fabsf(sks[d]));
-  #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ksmax = fmaxf(ksmax, __shfl_xor_sync(0xffffffffu, ksmax, o));
-    if (!isfinite(ksmax) && warp == 0 && lane == 0) record_error(a.err, PA_DEVERR_BAD_SCALE);
-    int e_kv = 0;
-    (void)frexpf(ksmax, &e_kv);
-    const float f_kv = ldexpf(1.f, -e_kv);
-
-    // Query operand.  Integer caches (INT8/INT4): q'' = 64 q' is split into four
-    // signed int8 digits, q'' = d0 + d1 2^-7 + d2 2^-14 + d3 2^-21 (residual below
-    // 2^-22), each digit a B operand of an exact int8 x int8 -> int32 MMA whose A
-    // operand is the raw cache code (INT4 as code + 8, corrected exactly with the
-    // digit sums).  FP8 caches: q' as an fp16 high part plus its fp16 residual.
-    // With LOPACK the second half of each pair rides in MMA columns 4..7.
-    uint32_t qf[NT][C::kQRegs];
-    float cw[NT][2][2];  // per accumulator column j: combine weights
-    int qoff[NT][2][2];  // per accumulator column j: integer offsets (magic - bias)
+    // ---- prologue: query fragments for this item (cooperative)
+    build_fragments<KV, D, BS, NT, LP>(a, smem + C::kQOff + slot * C::kQBytes, sks, nrows, frag,
+                                       rowc, tid);
+    consumer_sync();
+    uint32_t qf[NT][C::kQWords];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int k4 = 0; k4 < C::kQWords / 4; ++k4) {
+        const uint4 v = *reinterpret_cast<const uint4*>(
+            frag + (nt * 32 + lane) * C::kQStride + 4 * k4);
+        qf[nt][4 * k4 + 0] = v.x;
+        qf[nt][4 * k4 + 1] = v.y;
+        qf[nt][4 * k4 + 2] = v.z;
+        qf[nt][4 * k4 + 3] = v.w;
+      }
+    // per accumulator column j: logit weights and causal limit (LP: j = 0 only,
+    // the thread's row is tig)
+    float wA[NT][2], wB[NT][2];
     int lim[NT][2];
-    const __half* sq16 = reinterpret_cast<const __half*>(smem + C::kQOff + slot * C::kQBytes);
-    const __nv_bfloat16* sqbf = reinterpret_cast<const __nv_bfloat16*>(sq16);
-  #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int rl = LOPACK ? (g & 3) : nt * 8 + g;  // local row of B-operand column g
-      const bool valid = row0 + rl < row_end;
-      float w[C::kQElems];
-      float rmax = 0.f;
-  #pragma unroll
-      for (int i = 0; i < C::kQElems; ++i) {
-        const int ch = q_channel<KV>(i, tig);
-        float x = 0.f;
-        if (valid)
-          x = a.q_bf16 ? __bfloat162float(sqbf[rl * D + ch]) : __half2float(sq16[rl * D + ch]);
-        w[i] = x * (sks[ch] * f_kv);
-        rmax = fmaxf(rmax, fabsf(w[i]));
-      }
-      rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 1));
-      rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 2));
-      int e_q = 0;
-      (void)frexpf(rmax, &e_q);
-      const float c_mine = ldexpf(a.sm_scale_log2, e_kv + e_q);
-      if constexpr (C::kImma) {
-        const float f64 = ldexpf(1.f, 6 - e_q);
-        int dsum[4] = {0, 0, 0, 0};
-        uint32_t words[4][C::kQElems / 4];
-  #pragma unroll
-        for (int wd = 0; wd < C::kQElems / 4; ++wd)
-  #pragma unroll
-          for (int dg = 0; dg < 4; ++dg) words[dg][wd] = 0u;
-  #pragma unroll
-        for (int i = 0; i < C::kQElems; ++i) {
-          float r = w[i] * f64;  // |r| < 64
-          int dg_val[4];
-  #pragma unroll
-          for (int dg = 0; dg < 4; ++dg) {
-            const float dgt = rintf(r);
-            dg_val[dg] = static_cast<int>(dgt);
-            r = (r - dgt) * 128.f;
-          }
-  #pragma unroll
-          for (int dg = 0; dg < 4; ++dg) {
-            dsum[dg] += dg_val[dg];
-            words[dg][i / 4] |= (static_cast<uint32_t>(dg_val[dg]) & 0xFFu) << (8 * (i % 4));
-          }
-        }
-  #pragma unroll
-        for (int dg = 0; dg < 4; ++dg) {
-          dsum[dg] += __shfl_xor_sync(0xffffffffu, dsum[dg], 1);
-          dsum[dg] += __shfl_xor_sync(0xffffffffu, dsum[dg], 2);
-        }
-        // qf layout: [k32 step s][accumulator i][b register r]
-  #pragma unroll
-        for (int s = 0; s < D / 32; ++s)
-  #pragma unroll
-          for (int i = 0; i < C::kAcc; ++i)
-  #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-              // LOPACK: accumulator i carries digits (i=0: 0|1, i=1: 2|3), the odd
-              // digit in columns 4..7 (lanes with g >= 4)
-              const int dg = LOPACK ? (2 * i + (g >= 4 ? 1 : 0)) : i;
-              qf[nt][(s * C::kAcc + i) * 2 + r] = words[dg][s * 2 + r];
-            }
-        constexpr int kMagic = 0x4B400000;
-        const int kbias = (KV == PA_KV_INT4) ? 8 : 0;  // A operand holds code + 8
-  #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int col = 2 * tig + j;  // accumulator column held by this thread
-          const int src = col * 4;  // lanes with g = col supplied this column
-          if constexpr (LOPACK) {
-            // lane g = col supplied this column: digits 0|2 of row col (col < 4) or
-            // 1|3 of row col - 4; every lane holds all four digit sums of its row
-            const int sA = __shfl_sync(0xffffffffu, dsum[0], src);
-            const int sA1 = __shfl_sync(0xffffffffu, dsum[1], src);
-            const int sB = __shfl_sync(0xffffffffu, dsum[2], src);
-            const int sB1 = __shfl_sync(0xffffffffu, dsum[3], src);
-            const bool odd = col >= 4;
-            qoff[nt][j][0] = kMagic - kbias * (odd ? sA1 : sA);
-            qoff[nt][j][1] = kMagic - kbias * (odd ? sB1 : sB);
-            const int rr = col & 3;
-            const float cr = __shfl_sync(0xffffffffu, c_mine, rr * 4) * (1.f / 64.f);
-            // own value v = digit_even_or_odd + 2^-14 * next; S = v_even + 2^-7 v_odd
-            cw[nt][j][0] = odd ? cr * (1.f / 128.f) : cr;  // weight of own v
-            cw[nt][j][1] = odd ? cr : cr * (1.f / 128.f);  // weight of partner v
-          } else {
-            const int s0 = __shfl_sync(0xffffffffu, dsum[0], src);
-            const int s1 = __shfl_sync(0xffffffffu, dsum[1], src);
-            const int s2 = __shfl_sync(0xffffffffu, dsum[2], src);
-            const int s3 = __shfl_sync(0xffffffffu, dsum[3], src);
-            qoff[nt][j][0] = kbias * (s0 * 128 + s1);
-            qoff[nt][j][1] = kbias * (s2 * 128 + s3);
-            const float cr = __shfl_sync(0xffffffffu, c_mine, src) * (1.f / 64.f);
-            cw[nt][j][0] = cr * (1.f / 128.f);
-            cw[nt][j][1] = cr * (1.f / 2097152.f);  // 2^-21
-          }
-        }
-      } else {
-        const float f_q = ldexpf(1.f, -e_q);
-  #pragma unroll
-        for (int s = 0; s < D / 16; ++s) {
-          float hi[4], lo[4];
-  #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float xn = w[s * 4 + j] * f_q;
-            hi[j] = __half2float(__float2half_rn(xn));
-            lo[j] = xn - hi[j];
-          }
-          if constexpr (LOPACK) {
-            const bool use_lo = g >= 4;
-            qf[nt][s * 2 + 0] = pack_f32x2_to_h2(use_lo ? lo[0] : hi[0], use_lo ? lo[1] : hi[1]);
-            qf[nt][s * 2 + 1] = pack_f32x2_to_h2(use_lo ? lo[2] : hi[2], use_lo ? lo[3] : hi[3]);
-          } else {
-            qf[nt][s * 4 + 0] = pack_f32x2_to_h2(hi[0], hi[1]);
-            qf[nt][s * 4 + 1] = pack_f32x2_to_h2(hi[2], hi[3]);
-            qf[nt][s * 4 + 2] = pack_f32x2_to_h2(lo[0], lo[1]);
-            qf[nt][s * 4 + 3] = pack_f32x2_to_h2(lo[2], lo[3]);
-          }
-        }
-  #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int rr = LOPACK ? ((2 * tig + j) & 3) : 2 * tig + j;
-          cw[nt][j][0] = __shfl_sync(0xffffffffu, c_mine, rr * 4);
-          cw[nt][j][1] = 0.f;
-          qoff[nt][j][0] = qoff[nt][j][1] = 0;
-        }
-      }
-  #pragma unroll
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
       for (int j = 0; j < 2; ++j) {
-        const int rr = LOPACK ? ((2 * tig + j) & 3) : nt * 8 + 2 * tig + j;
-        lim[nt][j] = (row0 + rr < row_end && a.causal) ? past + (row0 + rr) / a.G : kmax - 1;
+        const int rl = LP ? tig : nt * 8 + 2 * tig + j;
+        const float cr = rowc[rl];
+        if constexpr (C::kInt) {
+          const float base = cr * ((KV == PA_KV_INT4) ? (1.f / 131072.f) : (1.f / 8192.f));
+          wA[nt][j] = base;                                            // C 2^-13 (/16 INT4)
+          wB[nt][j] = LP ? base * (1.f / 16384.f) : base * (1.f / 128.f);  // digits 2|3 or 2
+        } else {
+          wA[nt][j] = cr;
+          wB[nt][j] = 0.f;
+        }
+        lim[nt][j] = (row0 + rl < row_end && a.causal) ? past + (row0 + rl) / a.G : kmax - 1;
       }
-    }
+    consumer_sync();  // every warp holds its fragments: the area may be reused
 
     float o[NT][C::kMTiles][4];
-    float m_run[NT][2], l_run[NT][2];  // l_run: sum of the fp16-rounded P the MMA used
-  #pragma unroll
+    float lacc[NT][4];  // row sums of the fp16 P (ones-matrix MMA)
+    float m_run[NT][2], msub[NT][2], thr[NT][2];
+#pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-  #pragma unroll
+#pragma unroll
       for (int mt = 0; mt < C::kMTiles; ++mt)
-  #pragma unroll
+#pragma unroll
         for (int e = 0; e < 4; ++e) o[nt][mt][e] = 0.f;
-      m_run[nt][0] = m_run[nt][1] = -INFINITY;
-      l_run[nt][0] = l_run[nt][1] = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) lacc[nt][e] = 0.f;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        m_run[nt][j] = -INFINITY;
+        msub[nt][j] = 0.f;
+        thr[nt][j] = -INFINITY;
+      }
     }
-
-    // ldmatrix lane addressing: matrix (lane >> 3) covers rows (lane & 7) + 8 * (m & 1)
-    // of a 16-row key tile and chunk (2 cp + (m >> 1)).
-    const int lm = lane >> 3;
-    const int ld_row = (lane & 7) + 8 * (lm & 1);
-    const int ld_chunk = lm >> 1;
 
     for (int it = warp; alive && it * C::kBPI < nloc; it += C::kWarps) {
       const int lb0 = it * C::kBPI;
@@ -590,191 +744,255 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LOPACK>::kThreads)
       }
       if (!alive) break;
 
-      float x[C::kTPI][NT][4];  // logits (log2 units), then probabilities
-  #pragma unroll
+      // X: logits in log2 units minus the row's running reference, then P.
+      // LP: X[t][0][eh] = key g + 8 eh of row tig.  Else X[t][nt][e]: key g + 8 (e >> 1),
+      // row nt * 8 + 2 tig + (e & 1).
+      float X[C::kTPI][NT][4];
+#pragma unroll
       for (int t = 0; t < C::kTPI; ++t) {
         if (t >= ntiles) {
-  #pragma unroll
+#pragma unroll
           for (int nt = 0; nt < NT; ++nt)
-  #pragma unroll
-            for (int e = 0; e < 4; ++e) x[t][nt][e] = -INFINITY;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) X[t][nt][e] = -INFINITY;
           continue;
         }
         const int bi = t / C::kKeyTiles, kt = t % C::kKeyTiles;
         const uint32_t kbase = smem_u32(k_tile(warp * C::kSW + (kc + bi) % C::kSW));
         const int key0 = (blk_begin + lb0 + bi) * BS + kt * 16;
         const bool need_mask = key0 + 16 > kfull;
-        if constexpr (C::kImma) {
+        if constexpr (C::kInt) {
           int acc[C::kAcc][NT][4];
-  #pragma unroll
+#pragma unroll
           for (int i = 0; i < C::kAcc; ++i)
-  #pragma unroll
+#pragma unroll
             for (int nt = 0; nt < NT; ++nt)
-  #pragma unroll
+#pragma unroll
               for (int e = 0; e < 4; ++e) acc[i][nt][e] = 0;
-  #pragma unroll
+#pragma unroll
           for (int cp = 0; cp < C::kChunks / 2; ++cp) {
             uint32_t r[4];
             const uint32_t off = (kt * 16 + ld_row) * C::kCHS + (2 * cp + ld_chunk) * 16;
             ldsm_x4(kbase + swz<C::kSwzMask>(off), r);
-  #pragma unroll
+#pragma unroll
             for (int h = 0; h < (KV == PA_KV_INT4 ? 2 : 1); ++h) {
               uint32_t a0, a1, a2, a3;
               int s;
               if constexpr (KV == PA_KV_INT8) {
-                a0 = r[0]; a1 = r[1]; a2 = r[2]; a3 = r[3];  // 32 channels, no conversion
+                a0 = r[0]; a1 = r[1]; a2 = r[2]; a3 = r[3];  // 32 channels, raw codes
                 s = cp;
               } else {
-                const uint32_t x0 = r[2 * h], x1 = r[2 * h + 1];  // rows g, g+8 of chunk 2cp+h
-                a0 = i4lo_to_u8x4(x0);
-                a1 = i4lo_to_u8x4(x1);
-                a2 = i4hi_to_u8x4(x0);
-                a3 = i4hi_to_u8x4(x1);
+                // nibbles as signed bytes 16 x code: low nibbles shifted up, high masked
+                const uint32_t x0 = r[2 * h], x1 = r[2 * h + 1];  // keys g, g+8; chunk 2cp+h
+                a0 = (x0 << 4) & 0xF0F0F0F0u;
+                a1 = (x1 << 4) & 0xF0F0F0F0u;
+                a2 = x0 & 0xF0F0F0F0u;
+                a3 = x1 & 0xF0F0F0F0u;
                 s = 2 * cp + h;
               }
-  #pragma unroll
+#pragma unroll
               for (int nt = 0; nt < NT; ++nt)
-  #pragma unroll
+#pragma unroll
                 for (int i = 0; i < C::kAcc; ++i)
-                  imma_16832<KV == PA_KV_INT4>(acc[i][nt], a0, a1, a2, a3,
-                                               qf[nt][(s * C::kAcc + i) * 2],
-                                               qf[nt][(s * C::kAcc + i) * 2 + 1]);
+                  imma_16832<false>(acc[i][nt], a0, a1, a2, a3, qf[nt][(s * C::kAcc + i) * 2],
+                                    qf[nt][(s * C::kAcc + i) * 2 + 1]);
             }
           }
-  #pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-  #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int j = e & 1;
-              float xv;
-              if constexpr (LOPACK) {
-                const float f1 = int_to_float_exact(acc[0][nt][e], qoff[nt][j][0]);
-                const float f2 = int_to_float_exact(acc[1][nt][e], qoff[nt][j][1]);
-                const float v = fmaf(f2, 1.f / 16384.f, f1);
-                const float pv = __shfl_xor_sync(0xffffffffu, v, 2);
-                xv = fmaf(pv, cw[nt][j][1], v * cw[nt][j][0]);
-              } else {
-                const int A = acc[0][nt][e] * 128 + acc[1][nt][e] - qoff[nt][j][0];
-                const int B = acc[2][nt][e] * 128 + acc[3][nt][e] - qoff[nt][j][1];
-                xv = fmaf(__int2float_rn(B), cw[nt][j][1], __int2float_rn(A) * cw[nt][j][0]);
-              }
-              if (need_mask && key0 + g + (e >> 1) * 8 > lim[nt][j]) xv = -INFINITY;
-              x[t][nt][e] = xv;
+          if constexpr (LP) {
+#pragma unroll
+            for (int eh = 0; eh < 2; ++eh) {
+              const int A = acc[0][0][2 * eh] * 128 + acc[0][0][2 * eh + 1];
+              const int B2 = acc[1][0][2 * eh] * 128 + acc[1][0][2 * eh + 1];
+              float xv = fmaf(__int2float_rn(A), wA[0][0],
+                              fmaf(__int2float_rn(B2), wB[0][0], -msub[0][0]));
+              if (need_mask && key0 + g + 8 * eh > lim[0][0]) xv = -INFINITY;
+              X[t][0][eh] = xv;
             }
+          } else {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int j = e & 1;
+                const int A = acc[0][nt][e] * 128 + acc[1][nt][e];
+                float xv = fmaf(__int2float_rn(A), wA[nt][j],
+                                fmaf(__int2float_rn(acc[2][nt][e]), wB[nt][j], -msub[nt][j]));
+                if (need_mask && key0 + g + (e >> 1) * 8 > lim[nt][j]) xv = -INFINITY;
+                X[t][nt][e] = xv;
+              }
+          }
         } else {
-          float sacc[NT][4], sres[NT][4];
-  #pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-  #pragma unroll
-            for (int e = 0; e < 4; ++e) sacc[nt][e] = sres[nt][e] = 0.f;
-  #pragma unroll
+          float sacc[C::kAcc][NT][4];
+#pragma unroll
+          for (int i = 0; i < C::kAcc; ++i)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) sacc[i][nt][e] = 0.f;
+#pragma unroll
           for (int cp = 0; cp < C::kChunks / 2; ++cp) {
             uint32_t r[4];
             const uint32_t off = (kt * 16 + ld_row) * C::kCHS + (2 * cp + ld_chunk) * 16;
             ldsm_x4(kbase + swz<C::kSwzMask>(off), r);
-  #pragma unroll
+#pragma unroll
             for (int h = 0; h < 2; ++h) {
               const int s = 2 * cp + h;  // 16-channel k-step
               uint32_t a0, a1, a2, a3;
-              e4m3x4_to_h2x2(r[2 * h], a0, a2);      // row g: channels +0,1 | +2,3
-              e4m3x4_to_h2x2(r[2 * h + 1], a1, a3);  // row g+8
-  #pragma unroll
-              for (int nt = 0; nt < NT; ++nt) {
-                if constexpr (LOPACK) {
-                  mma_16816(sacc[nt], a0, a1, a2, a3, qf[nt][s * 2], qf[nt][s * 2 + 1]);
-                } else {
-                  mma_16816(sacc[nt], a0, a1, a2, a3, qf[nt][s * 4], qf[nt][s * 4 + 1]);
-                  mma_16816(sres[nt], a0, a1, a2, a3, qf[nt][s * 4 + 2], qf[nt][s * 4 + 3]);
-                }
-              }
+              e4m3x4_to_h2x2(r[2 * h], a0, a2);      // key g: channels +0,1 | +2,3
+              e4m3x4_to_h2x2(r[2 * h + 1], a1, a3);  // key g+8
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int i = 0; i < C::kAcc; ++i)
+                  mma_16816(sacc[i][nt], a0, a1, a2, a3, qf[nt][(s * C::kAcc + i) * 2],
+                            qf[nt][(s * C::kAcc + i) * 2 + 1]);
             }
           }
-  #pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-  #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int j = e & 1;
-              float sv = sacc[nt][e];
-              if constexpr (LOPACK)
-                sv += __shfl_xor_sync(0xffffffffu, sv, 2);  // high part + residual part
-              else
-                sv += sres[nt][e];
-              float xv = sv * cw[nt][j][0];
-              if (need_mask && key0 + g + (e >> 1) * 8 > lim[nt][j]) xv = -INFINITY;
-              x[t][nt][e] = xv;
+          if constexpr (LP) {
+#pragma unroll
+            for (int eh = 0; eh < 2; ++eh) {
+              // columns 2 tig / 2 tig + 1: high part / residual of row tig
+              float xv = fmaf(sacc[0][0][2 * eh] + sacc[0][0][2 * eh + 1], wA[0][0], -msub[0][0]);
+              if (need_mask && key0 + g + 8 * eh > lim[0][0]) xv = -INFINITY;
+              X[t][0][eh] = xv;
             }
+          } else {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int j = e & 1;
+                float xv = fmaf(sacc[0][nt][e] + sacc[1][nt][e], wA[nt][j], -msub[nt][j]);
+                if (need_mask && key0 + g + (e >> 1) * 8 > lim[nt][j]) xv = -INFINITY;
+                X[t][nt][e] = xv;
+              }
+          }
         }
       }
 
       // ---------------- online softmax with a lazily raised running max
-  #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-  #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          float lmx = -INFINITY;
-  #pragma unroll
-          for (int t = 0; t < C::kTPI; ++t) lmx = fmaxf(lmx, fmaxf(x[t][nt][j], x[t][nt][j + 2]));
-          const bool raise = lmx > m_run[nt][j] + 8.f;
-          if (__any_sync(0xffffffffu, raise)) {
-            lmx = fmaxf(lmx, __shfl_xor_sync(0xffffffffu, lmx, 4));
-            lmx = fmaxf(lmx, __shfl_xor_sync(0xffffffffu, lmx, 8));
-            lmx = fmaxf(lmx, __shfl_xor_sync(0xffffffffu, lmx, 16));
-            if (lmx > m_run[nt][j]) {
-              const float alpha = fast_exp2(m_run[nt][j] - lmx);  // 0 when m_run = -inf
-              m_run[nt][j] = lmx;
-              l_run[nt][j] *= alpha;
-  #pragma unroll
-              for (int mt = 0; mt < C::kMTiles; ++mt) {
-                o[nt][mt][j] *= alpha;
-                o[nt][mt][j + 2] *= alpha;
-              }
+      if constexpr (LP) {
+        float mx = fmaxf(fmaxf(X[0][0][0], X[0][0][1]), fmaxf(X[1][0][0], X[1][0][1]));
+        if (__any_sync(kFull, mx > thr[0][0])) {
+          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
+          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
+          if (mx > thr[0][0]) {
+            const float mnew = mx + msub[0][0];
+            const float alpha = (m_run[0][0] == -INFINITY) ? 0.f : fast_exp2(m_run[0][0] - mnew);
+#pragma unroll
+            for (int mt = 0; mt < C::kMTiles; ++mt)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) o[0][mt][e] *= alpha;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) lacc[0][e] *= alpha;
+#pragma unroll
+            for (int t = 0; t < C::kTPI; ++t) {
+              X[t][0][0] -= mx;
+              X[t][0][1] -= mx;
             }
-          }
-          const float m_ref = (m_run[nt][j] == -INFINITY) ? 0.f : m_run[nt][j];
-  #pragma unroll
-          for (int t = 0; t < C::kTPI; ++t) {
-            x[t][nt][j] = fast_exp2(x[t][nt][j] - m_ref);  // <= 2^8: safe range for fp16
-            x[t][nt][j + 2] = fast_exp2(x[t][nt][j + 2] - m_ref);
+            m_run[0][0] = mnew;
+            msub[0][0] = mnew;
+            thr[0][0] = 8.f;
           }
         }
+#pragma unroll
+        for (int t = 0; t < C::kTPI; ++t) {
+          X[t][0][0] = fast_exp2(X[t][0][0]);  // <= 2^8: safe range for fp16
+          X[t][0][1] = fast_exp2(X[t][0][1]);
+        }
+      } else {
+        float mx[NT][2];
+        bool any = false;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            mx[nt][j] = fmaxf(fmaxf(X[0][nt][j], X[0][nt][j + 2]),
+                              fmaxf(X[1][nt][j], X[1][nt][j + 2]));
+            any |= mx[nt][j] > thr[nt][j];
+          }
+        if (__any_sync(kFull, any)) {
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              float m = mx[nt][j];
+              m = fmaxf(m, __shfl_xor_sync(kFull, m, 4));
+              m = fmaxf(m, __shfl_xor_sync(kFull, m, 8));
+              m = fmaxf(m, __shfl_xor_sync(kFull, m, 16));
+              if (m > thr[nt][j]) {
+                const float mnew = m + msub[nt][j];
+                const float alpha =
+                    (m_run[nt][j] == -INFINITY) ? 0.f : fast_exp2(m_run[nt][j] - mnew);
+#pragma unroll
+                for (int mt = 0; mt < C::kMTiles; ++mt) {
+                  o[nt][mt][j] *= alpha;
+                  o[nt][mt][j + 2] *= alpha;
+                }
+                lacc[nt][j] *= alpha;
+                lacc[nt][j + 2] *= alpha;
+#pragma unroll
+                for (int t = 0; t < C::kTPI; ++t) {
+                  X[t][nt][j] -= m;
+                  X[t][nt][j + 2] -= m;
+                }
+                m_run[nt][j] = mnew;
+                msub[nt][j] = mnew;
+                thr[nt][j] = 8.f;
+              }
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < C::kTPI; ++t)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) X[t][nt][e] = fast_exp2(X[t][nt][e]);
       }
 
-      // ---------------- O^T[dim, row] += V^T P^T, per key tile
-  #pragma unroll
+      // ---------------- O^T[dim, col] += V^T P^T, per key tile
+#pragma unroll
       for (int t = 0; t < C::kTPI; ++t) {
         if (t >= ntiles) continue;
         const int bi = t / C::kKeyTiles, kt = t % C::kKeyTiles;
         const uint32_t vbase = smem_u32(v_tile(warp * C::kSW + (kc + bi) % C::kSW));
-        // P^T as the B operand: (key g; rows 2tig, 2tig+1) -> (keys 2tig, 2tig+1; row g);
-        // l_run accumulates exactly the fp16 values the MMA consumes.
         uint32_t pb[NT][2];
-  #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const uint32_t p01 = pack_f32x2_to_h2(x[t][nt][0], x[t][nt][1]);
-          const uint32_t p23 = pack_f32x2_to_h2(x[t][nt][2], x[t][nt][3]);
-          const __half2 h01 = u2h2(p01), h23 = u2h2(p23);
-          l_run[nt][0] += __low2float(h01) + __low2float(h23);
-          l_run[nt][1] += __high2float(h01) + __high2float(h23);
-          pb[nt][0] = movmatrix_trans(p01);
-          pb[nt][1] = movmatrix_trans(p23);
+        if constexpr (LP) {
+          // (row tig; keys g, g+8) -> column n = g: b0 (keys 2tig, 2tig+1) and b1
+          // (keys 2tig+8, 2tig+9) of row n / 2; movmatrix gives even lanes b0 and
+          // odd lanes b1, the partner lane (lane ^ 4) the other.
+          const uint32_t p = pack_f32x2_to_h2(X[t][0][0], X[t][0][1]);
+          const uint32_t mtr = movmatrix_trans(p);
+          const uint32_t y = __shfl_xor_sync(kFull, mtr, 4);
+          pb[0][0] = (g & 1) ? y : mtr;
+          pb[0][1] = (g & 1) ? mtr : y;
+        } else {
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            pb[nt][0] = movmatrix_trans(pack_f32x2_to_h2(X[t][nt][0], X[t][nt][1]));
+            pb[nt][1] = movmatrix_trans(pack_f32x2_to_h2(X[t][nt][2], X[t][nt][3]));
+          }
         }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          mma_16816(lacc[nt], kOnesH2, kOnesH2, kOnesH2, kOnesH2, pb[nt][0], pb[nt][1]);
         const int tkey0 = (blk_begin + lb0 + bi) * BS + kt * 16;
-  #pragma unroll
+#pragma unroll
         for (int cp = 0; cp < C::kChunks / 2; ++cp) {
           uint32_t r[4];
           const uint32_t off = (kt * 16 + ld_row) * C::kCHS + (2 * cp + ld_chunk) * 16;
           ldsm_x4_trans(vbase + swz<C::kSwzMask>(off), r);
-  #pragma unroll
+#pragma unroll
           for (int h = 0; h < 2; ++h) {
             const uint32_t lo = r[2 * h], hi = r[2 * h + 1];  // keys 2tig.. / 2tig+8.. of chunk c
             const int c = 2 * cp + h;
-  #pragma unroll
+#pragma unroll
             for (int hh = 0; hh < (KV == PA_KV_INT4 ? 2 : 1); ++hh) {
               uint32_t a0, a1, a2, a3;
               int mt;
               if constexpr (KV == PA_KV_INT8) {
-                // fp16 1024 + (code + 128): the constant 1152 per key is removed once
-                // at the end as 1152 * sum(P)
+                // fp16 1024 + (code + 128) = 1152 + code
                 const uint32_t ylo = lo ^ 0x80808080u, yhi = hi ^ 0x80808080u;
                 a0 = prmt(ylo, 0x64646464u, 0x4240);
                 a1 = prmt(ylo, 0x64646464u, 0x4341);
@@ -798,14 +1016,15 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LOPACK>::kThreads)
                 }
                 mt = c;
               } else {
-                const uint32_t zl = lo >> (8 * hh), zh = hi >> (8 * hh);
-                a0 = i4lo_to_h2(zl);
-                a1 = i4hi_to_h2(zl);
-                a2 = i4lo_to_h2(zh);
-                a3 = i4hi_to_h2(zh);
+                // low nibble: fp16 1024 + (code + 8); high nibble: 1024 + 16 (code + 8)
+                const uint32_t zl = hh ? (lo >> 8) : lo, zh = hh ? (hi >> 8) : hi;
+                a0 = (zl & 0x000F000Fu) ^ 0x64086408u;
+                a1 = (zl & 0x00F000F0u) ^ 0x64806480u;
+                a2 = (zh & 0x000F000Fu) ^ 0x64086408u;
+                a3 = (zh & 0x00F000F0u) ^ 0x64806480u;
                 mt = 2 * c + hh;
               }
-  #pragma unroll
+#pragma unroll
               for (int nt = 0; nt < NT; ++nt)
                 mma_16816(o[nt][mt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
             }
@@ -818,178 +1037,226 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LOPACK>::kThreads)
       kc += nb;
     }
 
-    // ======================================================== merge the warps
-    // Accumulator column 2 tig + j holds local row nt*8 + 2 tig + j (with LOPACK:
-    // row (2 tig + j) & 3, columns 4..7 duplicating rows 0..3, so only tig < 2
-    // writes).
-    const bool writer = !LOPACK || tig < 2;
-  #pragma unroll
+    // ---- this warp's result: remove the code->fp16 constants (using the exact
+    // row sums of P); columns j of the accumulators (LP: both = row tig)
+#pragma unroll
     for (int nt = 0; nt < NT; ++nt)
-  #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        float l = l_run[nt][j];
-        l += __shfl_xor_sync(0xffffffffu, l, 4);
-        l += __shfl_xor_sync(0xffffffffu, l, 8);
-        l += __shfl_xor_sync(0xffffffffu, l, 16);
-        l_run[nt][j] = l;
-        if (g == 0 && writer) {
-          sm_m[warp * C::kRows + nt * 8 + 2 * tig + j] = m_run[nt][j];
-          sm_l[warp * C::kRows + nt * 8 + 2 * tig + j] = l;
-        }
-      }
-    consumer_sync();
-    // The warps' rescaled outputs are summed into one [rows, D] buffer, warp 3
-    // first, then 2, 1, 0 (a fixed order: results are bitwise reproducible).
-    for (int wsum = C::kWarps - 1; wsum >= 0; --wsum) {
-      if (warp == wsum && writer) {
-  #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-  #pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int row = nt * 8 + 2 * tig + j;
-            float M = -INFINITY;
-  #pragma unroll
-            for (int w = 0; w < C::kWarps; ++w) M = fmaxf(M, sm_m[w * C::kRows + row]);
-            const float f = (m_run[nt][j] == -INFINITY) ? 0.f : fast_exp2(m_run[nt][j] - M);
-            // INT8 V entered the MMA as fp16 (1152 + code): remove 1152 * sum(P)
-            const float vbias = (KV == PA_KV_INT8) ? 1152.f * l_run[nt][j] : 0.f;
-  #pragma unroll
-            for (int mt = 0; mt < C::kMTiles; ++mt) {
-              const int d = out_dim<KV>(mt, g);
-              float2* dst = reinterpret_cast<float2*>(epi + row * D + d);
-              float2 v = make_float2((o[nt][mt][j] - vbias) * f, (o[nt][mt][j + 2] - vbias) * f);
-              if (wsum != C::kWarps - 1) {
-                const float2 prev = *dst;
-                v.x += prev.x;
-                v.y += prev.y;
-              }
-              *dst = v;
-            }
+#pragma unroll
+      for (int mt = 0; mt < C::kMTiles; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float l = lacc[nt][LP ? 0 : (e & 1)];
+          if constexpr (KV == PA_KV_INT8) {
+            o[nt][mt][e] = fmaf(-1152.f, l, o[nt][mt][e]);
+          } else if constexpr (KV == PA_KV_INT4) {
+            o[nt][mt][e] = (e < 2) ? fmaf(-1032.f, l, o[nt][mt][e])
+                                   : fmaf(-1152.f, l, o[nt][mt][e]) * (1.f / 16.f);
           }
-      }
+        }
+
+    // ---- merge the four warps' (m, l, O); warp 0 ends with the total.
+    // Slice rows are [row][D] fp32 with swizzled dim pairs.
+    auto slice_sw = [&](int row) { return LP ? (row & 3) : ((row >> 1) & 3); };
+    auto write_slice = [&](float* sl, float* ml) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int j = 0; j < (LP ? 1 : 2); ++j) {
+          const int row = LP ? tig : nt * 8 + 2 * tig + j;
+#pragma unroll
+          for (int mt = 0; mt < C::kMTiles; ++mt) {
+            const int dcol = slice_col(out_dim<KV>(mt, g), slice_sw(row));
+            *reinterpret_cast<float2*>(sl + row * D + dcol) =
+                make_float2(o[nt][mt][j], o[nt][mt][j + 2]);
+          }
+          if (g == 0) {
+            ml[row] = m_run[nt][j];
+            ml[C::kRows + row] = lacc[nt][LP ? 0 : j];
+          }
+        }
+    };
+    // Adds a slice (m_s, l_s, O_s) into this warp's (m, l, O).
+    auto merge_slice = [&](const float* sl, const float* ml) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int j = 0; j < (LP ? 1 : 2); ++j) {
+          const int row = LP ? tig : nt * 8 + 2 * tig + j;
+          const float ms = ml[row], ls = ml[C::kRows + row];
+          const float M = fmaxf(m_run[nt][j], ms);
+          const float fo = (m_run[nt][j] == -INFINITY) ? 0.f : fast_exp2(m_run[nt][j] - M);
+          const float fs = (ms == -INFINITY) ? 0.f : fast_exp2(ms - M);
+#pragma unroll
+          for (int mt = 0; mt < C::kMTiles; ++mt) {
+            const int dcol = slice_col(out_dim<KV>(mt, g), slice_sw(row));
+            const float2 v = *reinterpret_cast<const float2*>(sl + row * D + dcol);
+            o[nt][mt][j] = fmaf(v.x, fs, o[nt][mt][j] * fo);
+            o[nt][mt][j + 2] = fmaf(v.y, fs, o[nt][mt][j + 2] * fo);
+          }
+          const int jl = LP ? 0 : j;
+          lacc[nt][jl] = fmaf(ls, fs, lacc[nt][jl] * fo);
+          m_run[nt][j] = M;
+        }
+    };
+    if constexpr (LP) {
+      if (warp > 0) write_slice(slices + (warp - 1) * C::kSliceBytes / 4,
+                                sm_ml + (warp - 1) * 2 * C::kRows);
       consumer_sync();
+      if (warp == 0)
+#pragma unroll
+        for (int sl = 0; sl < C::kSlices; ++sl)
+          merge_slice(slices + sl * C::kSliceBytes / 4, sm_ml + sl * 2 * C::kRows);
+      consumer_sync();
+    } else {
+      for (int wsum = C::kWarps - 1; wsum >= 0; --wsum) {
+        if (warp == wsum) {
+          if (wsum != C::kWarps - 1) merge_slice(slices, sm_ml);
+          if (wsum != 0) write_slice(slices, sm_ml);
+        }
+        consumer_sync();
+      }
     }
 
-    const int nthr = C::kWarps * 32;
-    const int nrows = row_end - row0;
-    for (int idx = threadIdx.x; idx < nrows * (D / 2); idx += nthr) {
-      const int row = idx / (D / 2);
-      const int d = (idx % (D / 2)) * 2;
-      float M = -INFINITY;
-  #pragma unroll
-      for (int w = 0; w < C::kWarps; ++w) M = fmaxf(M, sm_m[w * C::kRows + row]);
-      float L = 0.f;
-  #pragma unroll
-      for (int w = 0; w < C::kWarps; ++w) {
-        const float mw = sm_m[w * C::kRows + row];
-        if (mw != -INFINITY) L += sm_l[w * C::kRows + row] * fast_exp2(mw - M);
+    // ---- warp 0: normalise, apply the V scale, store the output or the split partial
+    if (warp == 0) {
+      const bool is_split = nsplit > 1;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int j = 0; j < (LP ? 1 : 2); ++j) {
+          const int rl = LP ? tig : nt * 8 + 2 * tig + j;
+          if (rl >= nrows) continue;
+          const int r = row0 + rl;
+          const size_t orow = static_cast<size_t>(q0 + r / a.G) * a.H + kv * a.G + r % a.G;
+          const float L = lacc[nt][LP ? 0 : j];
+          const float inv = (L > 0.f) ? 1.f / L : 0.f;
+          const size_t prow = static_cast<size_t>(split) * a.total_q * a.H + orow;
+#pragma unroll
+          for (int mt = 0; mt < C::kMTiles; ++mt) {
+            const int dd = out_dim<KV>(mt, g);
+            const float2 vs = *reinterpret_cast<const float2*>(svs + dd);
+            const float o0 = o[nt][mt][j] * inv * vs.x;
+            const float o1 = o[nt][mt][j + 2] * inv * vs.y;
+            if (!is_split) {
+              if (a.out_bf16)
+                *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(a.out) +
+                                                   orow * D + dd) = __floats2bfloat162_rn(o0, o1);
+              else
+                *reinterpret_cast<__half2*>(reinterpret_cast<__half*>(a.out) + orow * D + dd) =
+                    __floats2half2_rn(o0, o1);
+            } else {
+              *reinterpret_cast<float2*>(a.o_part + prow * D + dd) = make_float2(o0, o1);
+            }
+          }
+          if (is_split && g == 0)
+            a.lse_part[prow] = (L > 0.f) ? m_run[nt][j] + __log2f(L) : -INFINITY;
+        }
+      if (is_split) {
+        // publish this split and count arrivals; the last split of the unit
+        // merges all of them and rewinds the counter for the next call
+        __threadfence();
+        __syncwarp();
+        uint32_t* counter =
+            a.counters + (static_cast<size_t>(b) * a.Hk + kv) * a.num_row_groups + rg;
+        int last = 0;
+        if (lane == 0) last = (atomicAdd(counter, 1u) == static_cast<uint32_t>(nsplit - 1));
+        last = __shfl_sync(kFull, last, 0);
+        if (lane == 0) *sm_flag = last;
       }
-      const float2 sv = *reinterpret_cast<const float2*>(epi + row * D + d);
-      const float s0 = sv.x, s1 = sv.y;
-      const float inv = (L > 0.f) ? 1.f / L : 0.f;
-      const float o0 = s0 * inv * svs[d];
-      const float o1 = s1 * inv * svs[d + 1];
-      const int r = row0 + row;
-      const size_t orow = static_cast<size_t>(q0 + r / a.G) * a.H + kv * a.G + r % a.G;
-      if (nsplit == 1) {
-        if (a.out_bf16)
-          *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(a.out) + orow * D +
-                                             d) = __floats2bfloat162_rn(o0, o1);
-        else
-          *reinterpret_cast<__half2*>(reinterpret_cast<__half*>(a.out) + orow * D + d) =
-              __floats2half2_rn(o0, o1);
-      } else {
-        const size_t prow = static_cast<size_t>(split) * a.total_q * a.H + orow;
-        *reinterpret_cast<float2*>(a.o_part + prow * D + d) = make_float2(o0, o1);
-        if (d == 0) a.lse_part[prow] = (L > 0.f) ? M + __log2f(L) : -INFINITY;
-      }
+      if (lane == 0 && !is_split) *sm_flag = 0;
     }
     if (nsplit > 1) {
-      // ---- split merge: publish this split and count arrivals; the last item
-      // of the unit merges all splits (log2-sum-exp weights) and rewinds the
-      // counter for the next call.
-      __threadfence();
-      consumer_sync();
-      uint32_t* counter =
-          a.counters + (static_cast<size_t>(b) * a.Hk + kv) * a.num_row_groups + rg;
-      if (threadIdx.x == 0) {
-        const uint32_t prev = atomicAdd(counter, 1u);
-        *sm_flag = (prev == static_cast<uint32_t>(nsplit - 1)) ? 1 : 0;
-      }
       consumer_sync();
       if (*sm_flag) {
         __threadfence();
         const size_t stride = static_cast<size_t>(a.total_q) * a.H;
         const int S = nsplit;
-        // 1) every (split, row) log2-sum-exp, loaded in parallel
-        for (int idx = threadIdx.x; idx < S * nrows; idx += nthr) {
+        const int nthr = C::kWarps * 32;
+        // 1) every (split, row) log2-sum-exp
+        for (int idx = tid; idx < S * nrows; idx += nthr) {
           const int s = idx / nrows, row = idx % nrows;
           const int r = row0 + row;
           const size_t orow = static_cast<size_t>(q0 + r / a.G) * a.H + kv * a.G + r % a.G;
           wts[s * C::kRows + row] = __ldcg(a.lse_part + s * stride + orow);
         }
         consumer_sync();
-        // 2) per row: weights 2^(lse_s - max) / sum
-        for (int row = threadIdx.x; row < nrows; row += nthr) {
+        // 2) per row (one warp per row): weights 2^(lse_s - max) / sum
+        for (int row = warp; row < nrows; row += C::kWarps) {
           float M = -INFINITY;
-          for (int s = 0; s < S; ++s) M = fmaxf(M, wts[s * C::kRows + row]);
+          for (int s = lane; s < S; s += 32) M = fmaxf(M, wts[s * C::kRows + row]);
+#pragma unroll
+          for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o2));
           float sum = 0.f;
-          for (int s = 0; s < S; ++s) {
+          for (int s = lane; s < S; s += 32) {
             const float ls = wts[s * C::kRows + row];
             const float wgt = (ls == -INFINITY) ? 0.f : fast_exp2(ls - M);
             wts[s * C::kRows + row] = wgt;
             sum += wgt;
           }
+#pragma unroll
+          for (int o2 = 16; o2 > 0; o2 >>= 1) sum += __shfl_xor_sync(kFull, sum, o2);
           const float inv = sum > 0.f ? 1.f / sum : 0.f;
-          for (int s = 0; s < S; ++s) wts[s * C::kRows + row] *= inv;
+          __syncwarp();
+          for (int s = lane; s < S; s += 32) wts[s * C::kRows + row] *= inv;
         }
         consumer_sync();
         // 3) weighted sum of the partials, eight splits in flight per thread
-        for (int idx = threadIdx.x; idx < nrows * (D / 2); idx += nthr) {
-          const int row = idx / (D / 2);
-          const int dd = (idx % (D / 2)) * 2;
+        for (int idx = tid; idx < nrows * (D / 4); idx += nthr) {
+          const int row = idx / (D / 4);
+          const int dd = (idx % (D / 4)) * 4;
           const int r = row0 + row;
           const size_t orow = static_cast<size_t>(q0 + r / a.G) * a.H + kv * a.G + r % a.G;
           const float* base = a.o_part + orow * D + dd;
-          float s0 = 0.f, s1 = 0.f;
+          float4 acc4 = make_float4(0.f, 0.f, 0.f, 0.f);
           for (int s8 = 0; s8 < S; s8 += 8) {
-            float2 v[8];
+            float4 v[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u)
               v[u] = (s8 + u < S)
-                         ? __ldcg(reinterpret_cast<const float2*>(base + (s8 + u) * stride * D))
-                         : make_float2(0.f, 0.f);
+                         ? __ldcg(reinterpret_cast<const float4*>(base + (s8 + u) * stride * D))
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
               if (s8 + u < S) {
                 const float wgt = wts[(s8 + u) * C::kRows + row];
-                s0 += wgt * v[u].x;
-                s1 += wgt * v[u].y;
+                acc4.x = fmaf(wgt, v[u].x, acc4.x);
+                acc4.y = fmaf(wgt, v[u].y, acc4.y);
+                acc4.z = fmaf(wgt, v[u].z, acc4.z);
+                acc4.w = fmaf(wgt, v[u].w, acc4.w);
               }
             }
           }
-          if (a.out_bf16)
-            *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(a.out) +
-                                               orow * D + dd) = __floats2bfloat162_rn(s0, s1);
-          else
-            *reinterpret_cast<__half2*>(reinterpret_cast<__half*>(a.out) + orow * D + dd) =
-                __floats2half2_rn(s0, s1);
+          if (a.out_bf16) {
+            __nv_bfloat162* dst =
+                reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(a.out) +
+                                                  orow * D + dd);
+            dst[0] = __floats2bfloat162_rn(acc4.x, acc4.y);
+            dst[1] = __floats2bfloat162_rn(acc4.z, acc4.w);
+          } else {
+            __half2* dst = reinterpret_cast<__half2*>(reinterpret_cast<__half*>(a.out) + orow * D + dd);
+            dst[0] = __floats2half2_rn(acc4.x, acc4.y);
+            dst[1] = __floats2half2_rn(acc4.z, acc4.w);
+          }
         }
-        if (threadIdx.x == 0) *counter = 0u;  // ready for the next call
+        if (tid == 0)
+          a.counters[(static_cast<size_t>(b) * a.Hk + kv) * a.num_row_groups + rg] = 0u;
       }
+      consumer_sync();  // weights / flag consumed before the next item's prologue
     }
     // the item slot (query rows, scales, descriptor) may be refilled
-    consumer_sync();
-    if (threadIdx.x == 0) mbar_arrive(item_empty(slot));
+    if (warp == 0) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(item_empty(slot));
+    }
     slot ^= 1;
   }
 }
 
-template <int KV, int D, int BS, int NT, bool LOPACK>
+template <int KV, int D, int BS, int NT, bool LP>
 static cudaError_t launch_t(const CUtensorMap& kmap, const CUtensorMap& vmap, FwdArgs a,
                             cudaStream_t stream) {
-  using C = Cfg<KV, D, BS, NT, LOPACK>;
-  auto kern = pa_fwd_kernel<KV, D, BS, NT, LOPACK>;
+  using C = Cfg<KV, D, BS, NT, LP>;
+  auto kern = pa_fwd_kernel<KV, D, BS, NT, LP>;
   // Per device: the dynamic shared-memory opt-in and the resident CTAs per SM.
   static std::atomic<int> ctas_per_sm[64] = {};
   int dev = 0;
@@ -1011,9 +1278,20 @@ static cudaError_t launch_t(const CUtensorMap& kmap, const CUtensorMap& vmap, Fw
   return cudaGetLastError();
 }
 
-template <int KV, int D, int BS, int NT, bool LOPACK>
+template <int KV, int D, int BS, int NT, bool LP>
 static int smem_t() {
-  return Cfg<KV, D, BS, NT, LOPACK>::kSmemBytes;
+  return Cfg<KV, D, BS, NT, LP>::kSmemBytes;
+}
+
+int forward_ctas_per_sm(int kv_dtype, int head_size, int block_size, int rows_per_cta) {
+  const int smem = forward_smem_bytes(kv_dtype, head_size, block_size, rows_per_cta);
+  if (smem <= 0) return 1;
+  // 228 KiB of shared memory per SM, 1 KiB reserved per CTA; the launch bounds
+  // cap registers at 3 CTAs (one n-tile) or 2 CTAs (two n-tiles) per SM.
+  int n = (228 * 1024) / (smem + 1024);
+  const int cap = rows_per_cta == 16 ? 2 : 3;
+  if (n > cap) n = cap;
+  return n < 1 ? 1 : n;
 }
 
 template <int KV, int D, int BS>

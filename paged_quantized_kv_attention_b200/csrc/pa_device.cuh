@@ -117,6 +117,11 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// Hint: bring the 128-byte line holding p into L2 (no fault for any address).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
+}
+
 // L2 policy for data that is read exactly once (the KV stream).
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   uint64_t p;

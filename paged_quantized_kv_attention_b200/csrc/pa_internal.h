@@ -18,18 +18,34 @@ struct FwdArgs {
   const int32_t* block_table;
   const int32_t* seqlens_k;
   const int32_t* cu_seqlens_q;
-  float* o_part;        // [num_splits, total_q * H, D] (split mode only)
-  float* lse_part;      // [num_splits, total_q * H] (log2 domain)
+  float* o_part;        // [max_splits, total_q * H, D] (split mode only)
+  float* lse_part;      // [max_splits, total_q * H] (log2 domain)
   uint32_t* counters;   // [batch * Hk * num_row_groups] split arrival counters (self-resetting)
   uint32_t* work;       // [2]: next work item, CTAs finished (both rewound by the last CTA)
   uint32_t* err;        // sticky device error word
   int batch, H, Hk, G, maxb, num_blocks, total_q;
   int q_bf16, out_bf16, causal;
-  int num_row_groups, num_splits, blocks_per_split;
-  int num_items;        // batch * Hk * num_row_groups * num_splits
-  int num_sms;          // SMs of the device (grid = resident CTAs per SM x num_sms)
+  int num_row_groups;   // largest number of row groups of a (sequence, KV head)
+  int max_splits;       // partial slots: no sequence is split into more items
+  int split_target;     // KV blocks per split target T: n blocks -> min(max_splits, ceil(n / T))
+                        // equal splits of ceil(n / splits) blocks
+  int num_items;        // work items of the plan (grid = min(num_items, resident CTAs))
+  int num_sms;          // SMs of the device
   float sm_scale_log2;  // softmax_scale * log2(e)
 };
+
+// Split geometry of a sequence with nblk KV blocks for split target T: the
+// number of non-empty splits and the blocks per split.  Shared by the planner
+// and the kernel so that both count the same items.
+__host__ __device__ inline void split_geometry(int nblk, int T, int max_splits, int* nsplit,
+                                               int* bps) {
+  int s = (nblk + T - 1) / T;
+  if (s < 1) s = 1;
+  if (s > max_splits) s = max_splits;
+  const int per = nblk > 0 ? (nblk + s - 1) / s : 1;
+  *bps = per;
+  *nsplit = nblk > 0 ? (nblk + per - 1) / per : 1;
+}
 
 // Workspace layout: [0, 256) header: error word at byte 0, work counters at
 // byte 64; then the split counters; then the partial outputs and their
@@ -44,6 +60,8 @@ cudaError_t launch_forward(int kv_dtype, int head_size, int block_size, int rows
                            cudaStream_t stream);
 // Dynamic shared memory of one forward CTA (-1 for an unsupported combination).
 int forward_smem_bytes(int kv_dtype, int head_size, int block_size, int rows_per_cta);
+// Forward CTAs resident per SM, from the launch bounds and shared memory.
+int forward_ctas_per_sm(int kv_dtype, int head_size, int block_size, int rows_per_cta);
 
 // Sets the thread's message for paged_attn_last_error() and returns st
 // (pa_api.cu; used by entry points defined in other files).

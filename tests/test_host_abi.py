@@ -67,14 +67,33 @@ def test_plan_zero_new_tokens_everywhere_is_a_no_op():
     pa.paged_attn_forward(None, None, None, None, None, None, None, None, None, p, stream=0)
 
 
+def _count_items(cu, L, G, Hk, bs, rows, T, max_splits):
+    """Work items by the documented split rule: a sequence with n KV blocks gets
+    s = min(max_splits, ceil(n / T)) splits of ceil(n / s) blocks (empty ones
+    dropped), times Hk KV heads times its row groups."""
+    total, most = 0, 1
+    for b in range(len(L)):
+        qb = int(cu[b + 1] - cu[b])
+        if qb == 0:
+            continue
+        n = -(-int(L[b]) // bs)
+        s = max(1, min(max_splits, -(-n // T)))
+        per = -(-n // s)
+        s = -(-n // per)
+        most = max(most, s)
+        total += Hk * (-(-qb * G // rows)) * s
+    return total, most
+
+
 @pytest.mark.parametrize("name,split", [("c1_tiny_int8", False), ("c2_int4_decode", True),
                                         ("c3_int8_long_split", True),
-                                        ("c4_ragged_prefill_int8", False),
-                                        ("c5_fp8_large_batch", True)])
+                                        ("c4_ragged_prefill_int8", None),
+                                        ("c5_fp8_large_batch", None)])
 def test_plan_split_decisions_on_the_workload_shapes(name, split):
-    """Flash-decoding split only when the units (B * Hk * row groups) give the
-    persistent CTAs (148 SMs x 3) fewer than 4 work items each, in splits of at
-    least 64 KB of K+V."""
+    """Flash-decoding split (the GQA GEMV decode page's rule, sized for the
+    resident CTAs): the tiny case stays whole, the cases whose (sequence, KV
+    head) units underfill the device are split, and the planned item count is
+    the documented split rule applied to the host lengths."""
     rng = np.random.default_rng(0)
     if name == "c1_tiny_int8":
         B, H, Hk, D, bs, L, ql = 2, 4, 1, 64, 16, np.array([37, 64]), np.ones(2, int)
@@ -95,13 +114,18 @@ def test_plan_split_decisions_on_the_workload_shapes(name, split):
     p = _params(batch=B, num_heads=H, kv_num_heads=Hk, head_size=D, block_size=bs,
                 num_blocks=maxb * B, max_blocks_per_seq=maxb, kv_dtype=kvd)
     ws = pa.paged_attn_plan(cu, L, p)
-    assert (p.num_splits > 1) == split
-    assert p.num_splits * p.blocks_per_split >= -(-int(L.max()) // bs)
+    if split is not None:
+        assert (p.num_splits > 1) == split
+    assert 1 <= p.num_splits <= 128 and p.blocks_per_split >= 1
+    items, most = _count_items(cu, L, H // Hk, Hk, bs, p.rows_per_cta, p.blocks_per_split, 128)
+    assert p.num_work_items == items
+    assert p.num_splits == most
     assert ws >= 256 and ws % 256 == 0
-    if split:
+    if p.num_splits > 1:
         assert ws >= 256 + p.num_splits * p.total_q * H * (D + 1) * 4
-        chs = D // 2 if name == "c2_int4_decode" else D
-        assert p.blocks_per_split * 2 * bs * chs >= 64 * 1024
+    if name == "c3_int8_long_split":
+        # equal sequences: one round of items over 148 SMs x 3 resident CTAs
+        assert p.num_work_items <= 148 * 3
 
 
 def test_plan_forced_and_disabled_split():
