@@ -130,8 +130,8 @@ typedef struct {
   /* ---- supplied by the caller before paged_attn_forward ---- */
   void* workspace;        /* device memory, 256-byte aligned, >= workspace_bytes,
                              zeroed once with paged_attn_workspace_init; holds the
-                             error word, the split arrival counters (they return to
-                             zero at the end of every call) and the split partials.
+                             error word, the work counters (they return to zero at
+                             the end of every call) and the split partials.
                              Calls that share a workspace must not overlap on the
                              GPU. */
   void* profile_events;   /* optional profiling hook: NULL, or a pointer to two
@@ -154,9 +154,10 @@ pa_status paged_attn_plan(const int32_t* cu_seqlens_q_host, const int32_t* seqle
 /* Attention forward (see the header comment for layouts).  params must come from
  * paged_attn_plan with the same lengths the device arrays hold.  total_q == 0
  * returns PA_OK without a launch.  Rows of sequences with q_b == 0 do not exist
- * in q/out; no other byte of out is written.  One kernel launch per call; when
- * params->num_splits > 1 the last CTA of each (sequence, KV head, row group)
- * merges the split partials (log-sum-exp) inside the same launch.  q, k_scale
+ * in q/out; no other byte of out is written.  One kernel launch per call, plus,
+ * when params->num_splits > 1, a log-sum-exp combine of the split partials
+ * launched as the forward kernel's programmatic dependent (it overlaps the
+ * forward kernel's tail and waits for its completion).  q, k_scale
  * and v_scale must be 16-byte aligned, the caches 16-byte aligned, out 4-byte
  * aligned.  After a device error the workspace should be re-initialised. */
 pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_cache,

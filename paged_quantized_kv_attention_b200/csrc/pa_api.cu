@@ -48,16 +48,17 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Workspace layout shared by the planner and the forward call.
 struct WsLayout {
-  size_t counters, o_part, lse_part, total;
+  size_t frag, o_part, lse_part, total;
 };
 
 WsLayout ws_layout(const paged_attn_params* p) {
   WsLayout w;
-  w.counters = kHeaderBytes;
   size_t off = kHeaderBytes;
+  w.frag = off;
+  const size_t units = static_cast<size_t>(p->batch) * p->kv_num_heads * p->num_row_groups;
+  const int uw = pa::fragment_unit_words(p->kv_dtype, p->head_size, p->rows_per_cta);
+  off = align256(off + units * static_cast<size_t>(uw > 0 ? uw : 0) * 4);
   if (p->num_splits > 1) {
-    const size_t units = static_cast<size_t>(p->batch) * p->kv_num_heads * p->num_row_groups;
-    off = align256(off + units * sizeof(uint32_t));
     w.o_part = off;
     const size_t rows = static_cast<size_t>(p->total_q) * p->num_heads;
     off = align256(off + rows * p->num_splits * p->head_size * sizeof(float));
@@ -135,18 +136,21 @@ pa_status get_encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
   return PA_OK;
 }
 
-// 3-D view of one cache pool: (cache_head_size bytes, kv_num_heads, num_blocks *
-// block_size tokens); the box is one block of one head.
+// 3-D view of one cache pool: (cache_head_size bytes, num_blocks * block_size
+// tokens, kv_num_heads); the box is 16 tokens of 4 heads, heads outermost in
+// shared memory so that each head's rows are contiguous there.
 pa_status encode_cache_map(const void* cache, const paged_attn_params* p, CUtensorMap* map) {
   PFN_cuTensorMapEncodeTiled_v12000 enc;
   pa_status st = get_encoder(&enc);
   if (st != PA_OK) return st;
   const int chs = cache_row_bytes(p->kv_dtype, p->head_size);
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(chs), static_cast<cuuint64_t>(p->kv_num_heads),
-                        static_cast<cuuint64_t>(p->num_blocks) * p->block_size};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(chs),
-                           static_cast<cuuint64_t>(chs) * p->kv_num_heads};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(chs), 1u, static_cast<cuuint32_t>(p->block_size)};
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(chs),
+                        static_cast<cuuint64_t>(p->num_blocks) * p->block_size,
+                        static_cast<cuuint64_t>(p->kv_num_heads)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(chs) * p->kv_num_heads,
+                           static_cast<cuuint64_t>(chs)};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(chs), 16u,
+                       static_cast<cuuint32_t>(pa::kHeadsPerItem)};
   cuuint32_t estr[3] = {1u, 1u, 1u};
   const CUtensorMapSwizzle swz = chs == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
                                  : chs == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
@@ -217,14 +221,16 @@ pa_status paged_attn_plan(const int32_t* cu_seqlens_q_host, const int32_t* seqle
   // Split target T (KV blocks per split).  Automatic choice: the T that minimises
   // an estimate of the makespan of the work items over the resident CTAs:
   // (rounds - 1) * mean item + largest item + rounds * per-item cost + the split
-  // partials' write and read spread over the CTAs + the final merge (latency
-  // and one CTA reading the partials) when anything is split (flash decoding after the
+  // partials' write and read spread over the CTAs + the combine kernel when
+  // anything is split (flash decoding after the
   // GQA GEMV decode page, Code analysis 2, sized for the resident CTA slots).
   const int rows = p->rows_per_cta;
-  const int Hk = p->kv_num_heads;
-  const double block_bytes = 2.0 * bs * cache_row_bytes(p->kv_dtype, p->head_size);
+  const int HP = pa::kHeadsPerItem;
+  const int Hg = (p->kv_num_heads + HP - 1) / HP;  // head groups: one item covers 4 KV heads
+  const double block_bytes = 2.0 * bs * cache_row_bytes(p->kv_dtype, p->head_size) *
+                             (p->kv_num_heads < HP ? p->kv_num_heads : HP);
   const double item_cost = kItemCostBytes / block_bytes;
-  const double part_cost = 2.0 * rows * p->head_size * 4.0 / block_bytes;
+  const double part_cost = 2.0 * HP * rows * p->head_size * 4.0 / block_bytes;
   const int64_t slots = static_cast<int64_t>(sms) *
                         pa::forward_ctas_per_sm(p->kv_dtype, p->head_size, bs, rows);
   auto count = [&](int T, int64_t* items, int64_t* split_items, int* max_bps, int* max_ns,
@@ -235,7 +241,7 @@ pa_status paged_attn_plan(const int32_t* cu_seqlens_q_host, const int32_t* seqle
     for (int b = 0; b < B; ++b) {
       const int qb = cu_seqlens_q_host[b + 1] - cu_seqlens_q_host[b];
       if (qb == 0) continue;
-      const int64_t units = static_cast<int64_t>(Hk) * ((static_cast<int64_t>(qb) * G + rows - 1) / rows);
+      const int64_t units = static_cast<int64_t>(Hg) * ((static_cast<int64_t>(qb) * G + rows - 1) / rows);
       const int nblk = (seqlens_k_host[b] + bs - 1) / bs;
       int ns, bps;
       pa::split_geometry(nblk, T, kMaxSplits, &ns, &bps);
@@ -262,11 +268,9 @@ pa_status paged_attn_plan(const int32_t* cu_seqlens_q_host, const int32_t* seqle
       count(Tc, &items, &split_items, &max_bps, &max_ns, &work);
       if (items <= 0) break;
       const int64_t rounds = (items + slots - 1) / slots;
-      // a split adds the last arrival's merge: its latency and its read of all
-      // the unit's partials by one CTA
+      // a split adds the combine kernel after the forward kernel
       const double est = (rounds - 1) * (work / items) + max_bps + rounds * item_cost +
-                         split_items * part_cost / slots +
-                         (max_ns > 1 ? 2.0 * item_cost + 0.5 * max_ns * part_cost : 0.0);
+                         split_items * part_cost / slots + (max_ns > 1 ? 2.0 * item_cost : 0.0);
       if (best < 0.0 || est < best) {
         best = est;
         T = Tc;
@@ -341,8 +345,8 @@ pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_c
   a.seqlens_k = seqlens_k;
   a.cu_seqlens_q = cu_seqlens_q;
   a.err = reinterpret_cast<uint32_t*>(ws);
-  a.counters = reinterpret_cast<uint32_t*>(ws + lay.counters);
   a.work = reinterpret_cast<uint32_t*>(ws + pa::kWsWorkOffset);
+  a.frag = reinterpret_cast<uint32_t*>(ws + lay.frag);
   a.o_part = p->num_splits > 1 ? reinterpret_cast<float*>(ws + lay.o_part) : nullptr;
   a.lse_part = p->num_splits > 1 ? reinterpret_cast<float*>(ws + lay.lse_part) : nullptr;
   a.batch = p->batch;
@@ -355,6 +359,7 @@ pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_c
   a.q_bf16 = p->q_dtype == PA_BF16;
   a.out_bf16 = p->out_dtype == PA_BF16;
   a.causal = p->causal;
+  a.rows_cta = p->rows_per_cta;
   a.num_row_groups = p->num_row_groups;
   a.max_splits = p->num_splits;
   a.split_target = p->blocks_per_split;
@@ -372,6 +377,10 @@ pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_c
   e = pa::launch_forward(p->kv_dtype, p->head_size, p->block_size, p->rows_per_cta, kmap, vmap,
                          a, s);
   if (e != cudaSuccess) return cuda_status(e, "forward launch");
+  if (p->num_splits > 1) {
+    e = pa::launch_combine(p->head_size, p->block_size, a, s);
+    if (e != cudaSuccess) return cuda_status(e, "combine launch");
+  }
   if (ev != nullptr && (e = cudaEventRecord(ev[1], s)) != cudaSuccess)
     return cuda_status(e, "profile event record");
   return ok();

@@ -1,40 +1,42 @@
 // pa_attention.cu -- fused paged quantised-KV GQA attention for sm_100a.
 //
-// Work items.  A unit is one (sequence, KV head, group of query rows): the rows
-// are the (new token, query head of the GQA group) pairs that read the same
-// keys.  They are the N side of the tensor-core tiles, keys the M side
-// ("swap-AB"), channels the K side.  A sequence with n KV blocks is split into
-// ceil(n / T) items of equal size (flash decoding), T chosen by the planner so
-// that the items fill the resident CTAs in whole rounds.  Items are numbered
-// densely over the sequences with new tokens: the producer warp of every CTA
-// computes the per-sequence item counts and their prefix sums once, from the
-// device lengths.  The kernel is persistent: CTA i starts with item i and then
-// pulls items from an atomic counter in the workspace.
+// Work items.  An item is (sequence, group of 4 KV heads, group of query rows,
+// KV split).  The rows of one head are the (new token, query head of the GQA
+// group) pairs that read that head's keys; they form the N side of the
+// tensor-core tiles, keys the M side ("swap-AB"), channels the K side.  A
+// sequence with n KV blocks is cut into ceil(n / T) equal splits (flash
+// decoding), T chosen by the planner so that the items fill the resident CTAs.
+// Items are numbered densely over the sequences with new tokens: the producer
+// warp of every CTA computes the per-sequence item counts and their prefix sums
+// once, from the device lengths.  The kernel is persistent: CTA i starts with
+// item i and then pulls items from an atomic counter in the workspace.
 //
-// Per CTA, one producer warp and four consumer warps:
-//   producer : per item, bulk-copies the query rows and both per-channel scale
-//              rows into one of two item slots, then streams the item's KV
-//              blocks (block table -> two 3-D TMA boxes per block: the K rows and
-//              the V rows of one head) into the consumers' stage rings, straight
-//              after the previous item's blocks.  The next item's index and block
-//              table entries are fetched while the current ones stream.
-//   consumers: per item, the four warps fold the K scale into the queries and
-//              encode them as B-operand fragments in shared memory (each warp a
-//              quarter of the work); then each warp takes alternate 32-key groups:
-//              ldmatrix (K) -> QK on the tensor cores -> online softmax (exp2
-//              domain, running maximum raised only when a logit exceeds it by more
-//              than 2^8) -> P^T in fp16 -> ldmatrix.trans (V) -> code -> fp16 ->
-//              PV MMA; finally the warps' (m, l, O) are merged through shared
-//              memory, the V scale applied once, and the result (or a split
-//              partial and its log2-sum-exp) stored.  The last split of a unit to
-//              finish merges the partials (arrival counter in the workspace).
+// Per CTA, one producer warp and four consumer warps, consumer warp w owning KV
+// head 4 hg + w of the item:
+//   producer : per item, bulk-copies the query rows and the k_scale rows of the
+//              four heads into the query buffer, then streams the item's KV in
+//              stages of 16 tokens: one 3-D TMA box (channels x 16 tokens x 4
+//              heads, heads outermost in shared memory) for K and one for V.
+//              Producer lane l owns ring stage l and refills it as soon as all
+//              four consumer warps have released it.
+//   consumers: per item, each warp folds its head's k_scale into its query rows
+//              and encodes them as B-operand fragments in registers, then for
+//              every stage: ldmatrix (its head's K rows) -> QK on the tensor cores
+//              -> online softmax (exp2 domain; the running maximum is raised only
+//              when a logit exceeds it by more than 2^8) -> P^T in fp16 ->
+//              ldmatrix.trans (V) -> code -> fp16 -> PV MMA.  At the end the warp
+//              applies the V scale and stores its head's rows, or writes a split
+//              partial and its log2-sum-exp; the last split of a (sequence, head,
+//              row group) to finish merges the partials (arrival counter in the
+//              workspace).  No consumer barrier: the warps never wait on each
+//              other.
 //
 // QK arithmetic.  INT8 and INT4 caches: the folded query q'' = q' 2^(6 - e_q)
 // (|q''| < 64) is split into signed int8 digits q'' = d0 + d1 2^-7 + d2 2^-14
 // (+ d3 2^-21), each the B operand of an exact mma.sync m16n8k32 s8 x s8 -> s32
 // whose A operand is the raw cache byte (INT4: the nibble shifted into the high
 // half of a byte, 16 x code).  FP8 caches: codes -> fp16 in registers, q' as an
-// fp16 high part plus an fp16 residual.  With at most 4 rows per item, MMA column
+// fp16 high part plus an fp16 residual.  With at most 4 rows per head, MMA column
 // n carries row n / 2, so a thread holds every digit (or both parts) of one row.
 // PV arithmetic.  V codes -> fp16 exactly with one byte permute (INT8:
 // 1152 + code) or one logic op (INT4: 1032 + code, 1152 + 16 code); the constant
@@ -61,76 +63,58 @@ namespace pa {
 constexpr uint32_t kFull = 0xffffffffu;
 constexpr uint32_t kOnesH2 = 0x3C003C00u;  // fp16x2 (1, 1)
 
-// NT: 8-column n-tiles per item (rows = 8 NT).  LP: at most 4 rows per item;
-// MMA column n carries row n / 2 (QK: the two halves of a digit/part pair;
-// PV: the row twice).
+// NT: 8-column n-tiles per head (rows = 8 NT).  LP: at most 4 rows per head; MMA
+// column n carries row n / 2 (QK: the two halves of a digit/part pair; PV: the
+// row twice).
 template <int KV, int D, int BS, int NT, bool LP>
 struct Cfg {
   static_assert(!LP || NT == 1, "row-pair packing uses one n-tile");
   static constexpr bool kInt = (KV != PA_KV_FP8_E4M3);
   static constexpr int kCHS = (KV == PA_KV_INT4) ? D / 2 : D;  // cache bytes per row
-  static constexpr int kTile = BS * kCHS;                       // one block, one head
-  static constexpr int kStageBytes = 2 * kTile;                 // K + V
+  static constexpr int kHP = kHeadsPerItem;                     // KV heads per item
+  static constexpr int kTok = 16;                               // tokens per stage
+  static constexpr int kSPB = BS / kTok;                        // stages per cache block
+  static constexpr int kHeadTile = kTok * kCHS;                 // one head's rows of a stage
+  static constexpr int kKTile = kHP * kHeadTile;                // K (or V) part of a stage
+  static constexpr int kStageBytes = 2 * kKTile;
   static constexpr int kChunks = kCHS / 16;                     // 16-byte chunks per row
   static constexpr int kSwzMask = (kCHS == 128) ? 7 : (kCHS == 64) ? 3 : 1;
   static constexpr int kMTiles = D / 16;                        // PV m-tiles (output dims)
-  static constexpr int kKeyTiles = BS / 16;                     // 16-key tiles per block
-  static constexpr int kBPI = (BS == 16) ? 2 : 1;               // blocks per warp iteration
-  static constexpr int kTPI = kBPI * kKeyTiles;                 // key tiles per iteration (2)
   static constexpr int kWarps = 4;                              // consumer warps
   static constexpr int kThreads = (kWarps + 1) * 32;            // + one producer warp
-  // ring: one sub-ring of kSW stages per consumer warp (fixed ownership), at
-  // least two iterations deep, about 64 KB in total
-  static constexpr int kSWRaw = 65536 / (kWarps * kStageBytes);
-  static constexpr int kSW = kSWRaw < 2 * kBPI ? 2 * kBPI : (kSWRaw > 16 ? 16 : kSWRaw);
-  static constexpr int kStages = kWarps * kSW;
-  // producer group: whole warp iterations, at most kSW blocks of any warp, <= 32 lanes
-  static constexpr int kItPerGroupRaw = (kSW < 8 ? kSW : 8) / kBPI;
-  static constexpr int kGroup = kWarps * kBPI * (kItPerGroupRaw < 1 ? 1 : kItPerGroupRaw);
-  static constexpr int kRows = LP ? 4 : 8 * NT;
+  static constexpr int kRows = LP ? 4 : 8 * NT;                 // query rows per head
   // QK accumulator sets per n-tile: integer digits (LP: 2 x 2 digits; else 3),
   // FP8 parts (LP: hi|lo in one; else hi, lo)
   static constexpr int kAcc = kInt ? (LP ? 2 : 3) : (LP ? 1 : 2);
   static constexpr int kDigits = LP ? 4 : 3;
   static constexpr int kKSteps = kInt ? D / 32 : D / 16;
   static constexpr int kQWords = kKSteps * kAcc * 2;            // B-fragment words per lane
-  static constexpr int kQStride =
-      ((kQWords / 4) % 2 == 0 && kQWords < 32) ? kQWords + 4 : kQWords;  // lds.128 banks
-  static constexpr int kUnits = D / 4;                          // 4-channel prologue units per row
-  static constexpr int kSlices = LP ? 3 : 1;                    // warp-merge buffers
   static constexpr int kMaxSplits = 128;
-  // shared memory map (offsets from the 1024-aligned base)
+  // Precomputed query fragments of one (sequence, KV head, row group) unit in
+  // the workspace: NT x 32 lanes x kQWords words (lane-major), then the kRows
+  // row logit multipliers, padded to 16 bytes.
+  static constexpr int kUnitWords = (NT * 32 * kQWords + kRows + 3) / 4 * 4;
+  // shared memory: the stage ring sized to the per-CTA budget (3 CTAs per SM with
+  // one n-tile, 2 with two)
+  static constexpr int kBudget = (NT == 1 ? 76800 : 115712) - 1024;
+  static constexpr int kStagesRaw = kBudget / kStageBytes;
+  static constexpr int kStages = kStagesRaw > 32 ? 32 : (kStagesRaw < 2 ? 2 : kStagesRaw);
   static constexpr int kRingBytes = kStages * kStageBytes;
-  static constexpr int kQBytes = kRows * D * 2;                 // query rows of one item slot
-  static constexpr int kQOff = kRingBytes;                      // 2 slots
-  static constexpr int kKsOff = kQOff + 2 * kQBytes;            // k_scale rows, 2 slots
-  static constexpr int kVsOff = kKsOff + 2 * D * 4;             // v_scale rows, 2 slots
-  static constexpr int kUnionOff = kVsOff + 2 * D * 4;          // fragments | merge slices | weights
-  static constexpr int kFragBytes = NT * 32 * kQStride * 4;
-  static constexpr int kSliceBytes = kRows * D * 4;
-  static constexpr int kWtsBytes = kMaxSplits * kRows * 4;
-  static constexpr int kU0 = kFragBytes > kSlices * kSliceBytes ? kFragBytes : kSlices * kSliceBytes;
-  static constexpr int kUnionBytes = kU0 > kWtsBytes ? kU0 : kWtsBytes;
-  static constexpr int kBarOff = kUnionOff + kUnionBytes;
-  static constexpr int kNumBars = 2 * kStages + 4;              // full, empty, item full/empty
+  static constexpr int kBarOff = kRingBytes;
+  static constexpr int kNumBars = 2 * kStages + 5;  // full, empty, item full/empty x2, fragments
   static constexpr int kDescOff = kBarOff + kNumBars * 8;
-  static constexpr int kMLOff = kDescOff + 2 * 64;              // merge m, l: [kSlices][2][kRows]
-  static constexpr int kCOff = kMLOff + kSlices * 2 * kRows * 4;  // row logit multipliers
-  static constexpr int kFlagOff = kCOff + kRows * 4;
-  static constexpr int kSmemBytes = kFlagOff + 16;
+  static constexpr int kSmemBytes = kDescOff + 2 * 64;
   static_assert(kChunks % 2 == 0, "ldmatrix.x4 covers two 16-byte chunks");
-  static_assert(kTile % ((kSwzMask + 1) * 128) == 0, "tiles keep the swizzle-atom alignment");
-  static_assert(kTPI == 2, "two 16-key tiles per warp iteration");
-  static_assert(kStages <= 64, "stage count");
-  static_assert(kGroup <= 32 && kGroup / (kWarps * kBPI) * kBPI <= kSW, "producer group");
-  static_assert(kQWords % 4 == 0 && kQStride % 4 == 0, "fragment rows are lds.128 aligned");
-  static_assert(kUnionOff % 16 == 0, "fragment area alignment");
+  static_assert(kHeadTile % ((kSwzMask + 1) * 128) == 0, "tiles keep the swizzle-atom alignment");
+  static_assert(kStages <= 32, "one producer lane per stage");
+  static_assert(BS % kTok == 0, "whole stages per block");
+  static_assert(kSmemBytes <= kBudget + 1024, "shared memory budget");
 };
 
 // One work item as published by the producer to the consumers (64 bytes).
 struct ItemDesc {
   int valid;  // 0: no more work
-  int b, kv, rg, split;
+  int b, hg, rg, split;
   int q0, row0, row_end, past, kmax, kfull;
   int blk_begin, nloc, Lb, nsplit, pad;
 };
@@ -148,8 +132,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-
-__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 // One bulk copy (global -> shared) completing on an mbarrier.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
@@ -169,9 +151,10 @@ __device__ __forceinline__ int out_dim(int mt, int g) {
   return 16 * mt + 2 * g;
 }
 
-// Column offset of dim pair d in a merge slice row (spreads the four row groups
-// of a warp over the banks).
-__device__ __forceinline__ int slice_col(int d, int sw) { return d ^ (sw << 3); }
+// Head groups of the device.
+__device__ __forceinline__ int head_groups(const FwdArgs& a) {
+  return (a.Hk + kHeadsPerItem - 1) / kHeadsPerItem;
+}
 
 // Items of sequence b (0 if it has no new tokens or its lengths are invalid).
 template <int BS>
@@ -187,7 +170,7 @@ __device__ __forceinline__ int seq_items(const FwdArgs& a, int rows_cta, int q0,
   }
   int ns, bps;
   split_geometry((Lb + BS - 1) / BS, a.split_target, a.max_splits, &ns, &bps);
-  return a.Hk * rg * ns;
+  return head_groups(a) * rg * ns;
 }
 
 // Rows, keys and block range of item `local` of sequence b.  Returns false (and
@@ -197,14 +180,14 @@ template <int BS>
 __device__ __forceinline__ bool decode_item(const FwdArgs& a, int rows_cta, int b, int local,
                                             int q0, int qb, int Lb, ItemDesc& d) {
   d.valid = 0;
-  const int R = qb * a.G;  // rows of (b, kv): row r = token r / G, head kv * G + r % G
+  const int R = qb * a.G;  // rows of (b, head): row r = token r / G, head h * G + r % G
   const int rg_n = (R + rows_cta - 1) / rows_cta;
   int ns, bps;
   split_geometry((Lb + BS - 1) / BS, a.split_target, a.max_splits, &ns, &bps);
   d.split = local % ns;
   const int rest = local / ns;
   d.rg = rest % rg_n;
-  d.kv = rest / rg_n;
+  d.hg = rest / rg_n;
   d.b = b;
   d.row0 = d.rg * rows_cta;
   d.row_end = min(R, d.row0 + rows_cta);
@@ -223,128 +206,165 @@ __device__ __forceinline__ bool decode_item(const FwdArgs& a, int rows_cta, int 
   return true;
 }
 
-// Blocks of an item with nloc blocks that consumer warp w takes: warp iterations
-// it = w, w + 4, ... each cover blocks it * BPI .. it * BPI + BPI - 1.
-template <int BPI>
-__device__ __forceinline__ int warp_blocks(int nloc, int w) {
-  const int full = nloc / (4 * BPI);
-  const int rem = nloc - full * 4 * BPI - w * BPI;
-  return full * BPI + (rem <= 0 ? 0 : (rem < BPI ? rem : BPI));
-}
-
 // ---------------------------------------------------------------------------
-// Query fragments.  The 128 consumer threads fold k_scale into the item's query
-// rows and write every lane's B-operand words to `frag` (lane-major, kQStride
-// words per lane), plus each row's logit multiplier C to `rowc`:
+// Query fragments of one head, built by one warp in registers.  Lane (g, tig)
+// folds k_scale into the channels its B-operand words carry for B column g and
+// encodes them; it also returns the logit multiplier C of that column's row:
 //   integer caches: logit (log2 units) = C 2^-6 sum_d code_d q''_d, q'' digits
 //   FP8           : logit = C sum_d code_d (hi_d + lo_d)
 // with C = softmax_scale log2(e) 2^(e_kv + e_q).
-// Word layout (per n-tile, per lane (g, tig)): word (s * kAcc + i) * 2 + r is
-// b-register r of k-step s for accumulator set i.  Channel of byte / half e:
+// Word (s * kAcc + i) * 2 + r is b-register r of k-step s for accumulator set i;
+// the channel of its byte / half e is
 //   INT8: 32 s + 16 r + 4 tig + e     INT4: 32 s + 8 tig + 2 e + r
-//   FP8 : 16 s + 4 tig + 2 r + e (e < 2, one fp16 per half)
-// These match the channels ldmatrix hands the same thread for the K operand.
+//   FP8 : 16 s + 4 tig + 2 r + e (e < 2)
+// matching the channels ldmatrix hands the same thread for the K operand.
+// B column g carries row g >> 1 (LP; digits / part g & 1) or row 8 nt + g.
+// qh: the query of the sequence's first new token, query head h * G (global);
+// row row0 + r of the (sequence, head) unit is token (row0 + r) / G, query head
+// h * G + (row0 + r) % G; sks: k_scale row of head h.
 template <int KV, int D, int BS, int NT, bool LP>
-__device__ __forceinline__ void build_fragments(const FwdArgs& a, const uint8_t* sq,
-                                                const float* sks, int nrows, uint32_t* frag,
-                                                float* rowc, int tid) {
+__device__ __forceinline__ void query_fragments(const FwdArgs& a, const uint8_t* qh,
+                                                const float* sks, int row0, int nrows, int lane,
+                                                uint32_t (&qf)[NT][Cfg<KV, D, BS, NT, LP>::kQWords],
+                                                float (&crow)[NT]) {
   using C = Cfg<KV, D, BS, NT, LP>;
-  const int lane = tid & 31;
+  const int g = lane >> 2, tig = lane & 3;
   float ksmax = 0.f;
 #pragma unroll
-  for (int d = lane; d < D; d += 32) ksmax = fmaxf(ksmax, fabsf(sks[d]));
+  for (int d = lane; d < D; d += 32) ksmax = fmaxf(ksmax, fabsf(__ldg(sks + d)));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ksmax = fmaxf(ksmax, __shfl_xor_sync(kFull, ksmax, o));
-  if (!isfinite(ksmax) && tid == 0) record_error(a.err, PA_DEVERR_BAD_SCALE);
+  if (!isfinite(ksmax) && lane == 0) record_error(a.err, PA_DEVERR_BAD_SCALE);
   int e_kv = 0;
   (void)frexpf(ksmax, &e_kv);
   const float f_kv = ldexpf(1.f, -e_kv);
-  const __half* q16 = reinterpret_cast<const __half*>(sq);
-  const __nv_bfloat16* qbf = reinterpret_cast<const __nv_bfloat16*>(sq);
-  constexpr int kU = C::kUnits;  // 32 (D = 128) or 16 lanes per row
-  for (int idx = tid; idx < C::kRows * kU; idx += 128) {
-    const int row = idx / kU, u = idx % kU;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int row = LP ? (g >> 1) : nt * 8 + g;
     const bool valid = row < nrows;
-    int s, r, tq, ch0, cstep;
-    if constexpr (KV == PA_KV_INT8) {
-      s = u >> 3; r = (u >> 2) & 1; tq = u & 3; ch0 = 32 * s + 16 * r + 4 * tq; cstep = 1;
-    } else if constexpr (KV == PA_KV_INT4) {
-      s = u >> 3; r = (u >> 2) & 1; tq = u & 3; ch0 = 32 * s + 8 * tq + r; cstep = 2;
-    } else {
-      s = u >> 2; r = 0; tq = u & 3; ch0 = 16 * s + 4 * tq; cstep = 1;
-    }
-    float w[4];
+    const int ru = row0 + row;
+    const size_t roff = valid ? (static_cast<size_t>(ru / a.G) * a.H + ru % a.G) * D : 0;
+    const __half* q16 = reinterpret_cast<const __half*>(qh) + roff;
+    const __nv_bfloat16* qbf = reinterpret_cast<const __nv_bfloat16*>(qh) + roff;
+    constexpr int kCh = 32;  // channels per lane (D = 128; 16 for D = 64)
+    constexpr int kN = D / 4;
+    float w[kN];
     float rmax = 0.f;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int ch = ch0 + e * cstep;
+    for (int i = 0; i < kN; ++i) {
+      int ch;
+      if constexpr (KV == PA_KV_INT8) {
+        const int s = i >> 3, r = (i >> 2) & 1, e = i & 3;
+        ch = 32 * s + 16 * r + 4 * tig + e;
+      } else if constexpr (KV == PA_KV_INT4) {
+        const int s = i >> 3, r = (i >> 2) & 1, e = i & 3;
+        ch = 32 * s + 8 * tig + 2 * e + r;
+      } else {
+        const int s = i >> 2, r = (i >> 1) & 1, e = i & 1;
+        ch = 16 * s + 4 * tig + 2 * r + e;
+      }
       float x = 0.f;
-      if (valid) x = a.q_bf16 ? __bfloat162float(qbf[row * D + ch]) : __half2float(q16[row * D + ch]);
-      w[e] = x * (sks[ch] * f_kv);
-      rmax = fmaxf(rmax, fabsf(w[e]));
+      if (valid) x = a.q_bf16 ? __bfloat162float(qbf[ch]) : __half2float(q16[ch]);
+      w[i] = x * (__ldg(sks + ch) * f_kv);
+      rmax = fmaxf(rmax, fabsf(w[i]));
     }
-#pragma unroll
-    for (int o = kU / 2; o > 0; o >>= 1) rmax = fmaxf(rmax, __shfl_xor_sync(kFull, rmax, o));
+    (void)kCh;
+    rmax = fmaxf(rmax, __shfl_xor_sync(kFull, rmax, 1));
+    rmax = fmaxf(rmax, __shfl_xor_sync(kFull, rmax, 2));
     int e_q = 0;
     (void)frexpf(rmax, &e_q);
-    if (u == 0) rowc[row] = ldexpf(a.sm_scale_log2, e_kv + e_q);
-    const int nt = LP ? 0 : row >> 3;
-    uint32_t* fr = frag + nt * 32 * C::kQStride;
+    crow[nt] = ldexpf(a.sm_scale_log2, e_kv + e_q);
     if constexpr (C::kInt) {
       const float f = ldexpf(1.f, 6 - e_q);
-      uint32_t wd[C::kDigits];
+      const int p = g & 1;
 #pragma unroll
-      for (int dg = 0; dg < C::kDigits; ++dg) wd[dg] = 0u;
+      for (int wd = 0; wd < kN / 4; ++wd) {  // word (s, r): elements 4 wd .. 4 wd + 3
+        uint32_t dg[C::kDigits];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float v = w[e] * f;  // |v| < 64; each remainder times 128 stays within +-64
+        for (int k = 0; k < C::kDigits; ++k) dg[k] = 0u;
 #pragma unroll
-        for (int dg = 0; dg < C::kDigits; ++dg) {
-          const float t = rintf(v);
-          wd[dg] |= (static_cast<uint32_t>(static_cast<int>(t)) & 0xFFu) << (8 * e);
-          v = (v - t) * 128.f;
+        for (int e = 0; e < 4; ++e) {
+          float v = w[4 * wd + e] * f;  // |v| < 64; each remainder times 128 stays within +-64
+#pragma unroll
+          for (int k = 0; k < C::kDigits; ++k) {
+            const float t = rintf(v);
+            dg[k] |= (static_cast<uint32_t>(static_cast<int>(t)) & 0xFFu) << (8 * e);
+            v = (v - t) * 128.f;
+          }
         }
-      }
-      if constexpr (LP) {
-        // column n = 2 row + p: set i carries digit 2 i + p
+        const int s = wd >> 1, r = wd & 1;
+        if constexpr (LP) {
+          // set i carries digit 2 i + p (p = g & 1)
+          qf[nt][(s * 2 + 0) * 2 + r] = p ? dg[1] : dg[0];
+          qf[nt][(s * 2 + 1) * 2 + r] = p ? dg[3] : dg[2];
+        } else {
 #pragma unroll
-        for (int p = 0; p < 2; ++p) {
-          uint32_t* fl = fr + ((2 * row + p) * 4 + tq) * C::kQStride;
-#pragma unroll
-          for (int i = 0; i < 2; ++i) fl[(s * 2 + i) * 2 + r] = wd[2 * i + p];
+          for (int i = 0; i < 3; ++i) qf[nt][(s * 3 + i) * 2 + r] = dg[i];
         }
-      } else {
-        uint32_t* fl = fr + ((row & 7) * 4 + tq) * C::kQStride;
-#pragma unroll
-        for (int i = 0; i < 3; ++i) fl[(s * 3 + i) * 2 + r] = wd[i];
       }
     } else {
       const float f = ldexpf(1.f, -e_q);
-      float hi[4], lo[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float xn = w[e] * f;  // |xn| < 1
-        hi[e] = __half2float(__float2half_rn(xn));
-        lo[e] = xn - hi[e];
-      }
-      const uint32_t h01 = pack_f32x2_to_h2(hi[0], hi[1]), h23 = pack_f32x2_to_h2(hi[2], hi[3]);
-      const uint32_t l01 = pack_f32x2_to_h2(lo[0], lo[1]), l23 = pack_f32x2_to_h2(lo[2], lo[3]);
-      if constexpr (LP) {
-        // column n = 2 row + p: part p (0 high, 1 residual)
-        uint32_t* f0 = fr + ((2 * row) * 4 + tq) * C::kQStride;
-        uint32_t* f1 = fr + ((2 * row + 1) * 4 + tq) * C::kQStride;
-        f0[s * 2 + 0] = h01;
-        f0[s * 2 + 1] = h23;
-        f1[s * 2 + 0] = l01;
-        f1[s * 2 + 1] = l23;
-      } else {
-        uint32_t* fl = fr + ((row & 7) * 4 + tq) * C::kQStride;
-        fl[(s * 2 + 0) * 2 + 0] = h01;
-        fl[(s * 2 + 0) * 2 + 1] = h23;
-        fl[(s * 2 + 1) * 2 + 0] = l01;
-        fl[(s * 2 + 1) * 2 + 1] = l23;
+      for (int wd = 0; wd < kN / 2; ++wd) {  // word (s, r): elements 2 wd, 2 wd + 1
+        const float x0 = w[2 * wd] * f, x1 = w[2 * wd + 1] * f;  // |x| < 1
+        const float h0 = __half2float(__float2half_rn(x0)), h1 = __half2float(__float2half_rn(x1));
+        const uint32_t hi = pack_f32x2_to_h2(h0, h1);
+        const uint32_t lo = pack_f32x2_to_h2(x0 - h0, x1 - h1);
+        const int s = wd >> 1, r = wd & 1;
+        if constexpr (LP) {
+          qf[nt][s * 2 + r] = (g & 1) ? lo : hi;  // column g: part g & 1
+        } else {
+          qf[nt][(s * 2 + 0) * 2 + r] = hi;
+          qf[nt][(s * 2 + 1) * 2 + r] = lo;
+        }
       }
     }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Fragment pre-pass: one warp per (sequence, KV head, row group) unit folds the
+// K scale into the unit's query rows and stores every lane's B-operand words and
+// the rows' logit multipliers in the workspace (query_fragments above), once per
+// unit instead of once per split item.  The forward kernel is launched as this
+// grid's programmatic dependent: it starts streaming KV right away and waits
+// for this grid only before its consumers load fragments.  Two warps per CTA, so
+// that a CTA fits beside three forward CTAs on one SM.
+template <int KV, int D, int BS, int NT, bool LP>
+__global__ void __launch_bounds__(64) pa_prep_kernel(const FwdArgs a) {
+  using C = Cfg<KV, D, BS, NT, LP>;
+  asm volatile("griddepcontrol.launch_dependents;");
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2, tig = lane & 3;
+  const long long units = static_cast<long long>(a.batch) * a.Hk * a.num_row_groups;
+  const long long u = static_cast<long long>(blockIdx.x) * 2 + (threadIdx.x >> 5);
+  if (u >= units) return;
+  const int rg = static_cast<int>(u % a.num_row_groups);
+  const int h = static_cast<int>((u / a.num_row_groups) % a.Hk);
+  const int b = static_cast<int>(u / (static_cast<long long>(a.num_row_groups) * a.Hk));
+  const int q0 = __ldg(a.cu_seqlens_q + b), qb = __ldg(a.cu_seqlens_q + b + 1) - q0;
+  const int Lb = __ldg(a.seqlens_k + b);
+  if (qb <= 0 || qb > Lb || q0 < 0 || q0 + qb > a.total_q) return;
+  const int R = qb * a.G;
+  const int row0 = rg * C::kRows;
+  if (row0 >= R) return;
+  const int nrows = min(R, row0 + C::kRows) - row0;
+  uint32_t qf[NT][C::kQWords];
+  float crow[NT];
+  const uint8_t* qh = reinterpret_cast<const uint8_t*>(a.q) +
+                      (static_cast<size_t>(q0) * a.H + static_cast<size_t>(h) * a.G) * D * 2;
+  query_fragments<KV, D, BS, NT, LP>(a, qh, a.k_scale + static_cast<size_t>(h) * D, row0, nrows,
+                                     lane, qf, crow);
+  uint32_t* fb = a.frag + static_cast<size_t>(u) * C::kUnitWords;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+    for (int k4 = 0; k4 < C::kQWords / 4; ++k4)
+      reinterpret_cast<uint4*>(fb + (nt * 32 + lane) * C::kQWords)[k4] =
+          make_uint4(qf[nt][4 * k4], qf[nt][4 * k4 + 1], qf[nt][4 * k4 + 2], qf[nt][4 * k4 + 3]);
+    // the lane of B column g holds the multiplier of row g >> 1 (LP) or 8 nt + g
+    if (tig == 0 && (!LP || (g & 1) == 0))
+      reinterpret_cast<float*>(fb + NT * 32 * C::kQWords)[LP ? (g >> 1) : nt * 8 + g] = crow[nt];
   }
 }
 
@@ -366,12 +386,6 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
   }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   ItemDesc* descs = reinterpret_cast<ItemDesc*>(smem + C::kDescOff);
-  float* sm_ml = reinterpret_cast<float*>(smem + C::kMLOff);
-  float* rowc = reinterpret_cast<float*>(smem + C::kCOff);
-  int* sm_flag = reinterpret_cast<int*>(smem + C::kFlagOff);
-  uint32_t* frag = reinterpret_cast<uint32_t*>(smem + C::kUnionOff);
-  float* slices = reinterpret_cast<float*>(smem + C::kUnionOff);
-  float* wts = slices;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -382,18 +396,25 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
   auto empty_bar = [&](int s) { return smem_u32(bars + C::kStages + s); };
   auto item_full = [&](int sl) { return smem_u32(bars + 2 * C::kStages + sl); };
   auto item_empty = [&](int sl) { return smem_u32(bars + 2 * C::kStages + 2 + sl); };
+  // completes once every consumer warp holds its first item's query fragments
+  const uint32_t frag_ready = smem_u32(bars + 2 * C::kStages + 4);
   auto k_tile = [&](int s) { return smem + s * C::kStageBytes; };
-  auto v_tile = [&](int s) { return smem + s * C::kStageBytes + C::kTile; };
+  auto v_tile = [&](int s) { return smem + s * C::kStageBytes + C::kKTile; };
 
+  // The combine kernel (launched after this one when the plan splits the KV)
+  // may be scheduled onto SMs as this grid's CTAs finish; it waits for this
+  // grid's completion before reading anything.
+  asm volatile("griddepcontrol.launch_dependents;");
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
+      mbar_init(empty_bar(s), C::kWarps);
     }
     for (int sl = 0; sl < 2; ++sl) {
       mbar_init(item_full(sl), 1);
-      mbar_init(item_empty(sl), 1);
+      mbar_init(item_empty(sl), C::kWarps);
     }
+    mbar_init(frag_ready, C::kWarps);
     mbar_fence_init();
   }
   __syncthreads();
@@ -465,8 +486,7 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
       }
       if (bad_any) record_error(a.err, PA_DEVERR_BAD_LENGTH);
     } else {
-      const int max_rg = a.num_row_groups;
-      per_seq = a.Hk * max_rg * a.max_splits;
+      per_seq = head_groups(a) * a.num_row_groups * a.max_splits;
       total = a.batch * per_seq;
     }
 
@@ -503,27 +523,22 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
         if (bad) record_error(a.err, PA_DEVERR_BAD_LENGTH);
         return false;
       }
-      int local = w - b * per_seq;
-      // sparse layout: split fastest over max_splits, then row group, then head
+      const int local = w - b * per_seq;
+      // sparse layout: split fastest over max_splits, then row group, then head group
       const int split = local % a.max_splits;
       const int rest = local / a.max_splits;
-      const int rg = rest % a.num_row_groups, kv = rest / a.num_row_groups;
+      const int rg = rest % a.num_row_groups, hg = rest / a.num_row_groups;
       const int R = qb * a.G;
       const int rg_n = (R + rows_cta - 1) / rows_cta;
       int ns, bps;
       split_geometry((Lb + BS - 1) / BS, a.split_target, a.max_splits, &ns, &bps);
       if (rg >= rg_n || split >= ns) return false;
-      return decode_item<BS>(a, rows_cta, b, (kv * rg_n + rg) * ns + split, q0, qb, Lb, d);
+      return decode_item<BS>(a, rows_cta, b, (hg * rg_n + rg) * ns + split, q0, qb, Lb, d);
     };
 
     int uses[2] = {0, 0};
     int slot = 0;
-    // Blocks handed to each consumer warp so far: warp w's k-th block lives in
-    // stage w * kSW + k % kSW of its own sub-ring, round k / kSW.
-    int cnt_w0 = 0, cnt_w1 = 0, cnt_w2 = 0, cnt_w3 = 0;
-    auto cnt_of = [&](int wq) {
-      return wq == 0 ? cnt_w0 : (wq == 1 ? cnt_w1 : (wq == 2 ? cnt_w2 : cnt_w3));
-    };
+    int done = 0;  // stages issued so far: item stage kk lands in ring stage (done + kk) % kStages
     bool ok = true;
     int w = blockIdx.x;  // first item without an atomic
     uint32_t w_pref = 0;
@@ -539,10 +554,21 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
         if (locate(w, d)) break;
         w = next_index();
       }
-      // block-table entries of the item's first group, fetched with the publish
       const int32_t* bt = a.block_table + static_cast<size_t>(d.b) * a.maxb + d.blk_begin;
-      int phys_cur = 0;
-      if (d.valid && lane < C::kGroup && lane < d.nloc) phys_cur = __ldg(bt + lane);
+      const int nst = d.valid ? d.nloc * C::kSPB : 0;
+      // Lane l < kStages owns ring stage l and issues the item's stages kk with
+      // (done + kk) % kStages == l, in order; first its block-table entry.
+      const bool owner = lane < C::kStages;
+      int kk = owner ? ((lane - done) % C::kStages + C::kStages) % C::kStages : 0;
+      auto load_phys = [&](int kq) {
+        int ph = __ldg(bt + kq / C::kSPB);
+        if (ph < 0 || ph >= a.num_blocks) {
+          record_error(a.err, PA_DEVERR_BAD_BLOCK);
+          ph = a.num_blocks;  // out-of-range box: TMA fills zeros, nothing faults
+        }
+        return ph;
+      };
+      int phys = (owner && kk < nst) ? load_phys(kk) : 0;
       // publish the item (or the end marker) in the next slot
       if (lane == 0) {
         if (uses[slot] > 0 && !mbar_wait(item_empty(slot), (uses[slot] - 1) & 1)) {
@@ -550,90 +576,79 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
           ok = false;
         } else {
           descs[slot] = d;
-          if (d.valid) {
-            const uint32_t row_bytes = D * 2;
-            const uint32_t tot =
-                static_cast<uint32_t>(d.row_end - d.row0) * row_bytes + 2 * D * 4;
-            mbar_arrive_expect_tx(item_full(slot), tot);
-            const int i_first = d.row0 / a.G, i_last = (d.row_end - 1) / a.G;
-            for (int i = i_first; i <= i_last; ++i) {
-              const int r_lo = max(d.row0, i * a.G), r_hi = min(d.row_end, (i + 1) * a.G);
-              const uint8_t* src = reinterpret_cast<const uint8_t*>(a.q) +
-                                   ((static_cast<size_t>(d.q0 + i) * a.H + d.kv * a.G +
-                                     (r_lo - i * a.G)) * D) * 2;
-              bulk_load(smem_u32(smem + C::kQOff + slot * C::kQBytes + (r_lo - d.row0) * row_bytes),
-                        src, static_cast<uint32_t>(r_hi - r_lo) * row_bytes, item_full(slot));
-            }
-            bulk_load(smem_u32(smem + C::kKsOff + slot * D * 4), a.k_scale + d.kv * D, D * 4,
-                      item_full(slot));
-            bulk_load(smem_u32(smem + C::kVsOff + slot * D * 4), a.v_scale + d.kv * D, D * 4,
-                      item_full(slot));
-          } else {
-            mbar_arrive(item_full(slot));
-          }
+          mbar_arrive(item_full(slot));
         }
       }
       ok = __shfl_sync(kFull, ok, 0);
       ++uses[slot];
       if (!ok || !d.valid) break;
 
-      // Blocks go out in groups of kGroup (whole warp iterations, at most kSW
-      // blocks of any warp, so every block of a group has its own stage): lane j
-      // waits for its stage to be released, arms it and issues the two boxes, all
-      // lanes in parallel; the next group's block-table entries are loaded first.
-      // Item block lb belongs to warp (lb / kBPI) % 4, the split the consumers use.
-      constexpr int kGroup = C::kGroup;
-      for (int base = 0; base < d.nloc && ok; base += kGroup) {
-        const int lb = base + lane;
-        int phys_nxt = 0;
-        if (lane < kGroup && lb + kGroup < d.nloc) phys_nxt = __ldg(bt + lb + kGroup);
-        bool mine_ok = true;
-        if (lane < kGroup && lb < d.nloc) {
-          int phys = phys_cur;
-          if (phys < 0 || phys >= a.num_blocks) {
-            record_error(a.err, PA_DEVERR_BAD_BLOCK);
-            phys = a.num_blocks;  // out-of-range box: TMA fills zeros, nothing faults
-          }
-          const int wq = (lb / C::kBPI) % C::kWarps;
-          const int k = cnt_of(wq) + (lb / (C::kWarps * C::kBPI)) * C::kBPI + lb % C::kBPI;
-          const int s = wq * C::kSW + k % C::kSW;
-          const int round = k / C::kSW;
-          if (round > 0 && !mbar_wait(empty_bar(s), (round - 1) & 1)) {
-            mine_ok = false;
-          } else {
-            mbar_arrive_expect_tx(full_bar(s), C::kStageBytes);
-            tma_load_3d(smem_u32(k_tile(s)), &kmap, full_bar(s), 0, d.kv, phys * BS, policy);
-            tma_load_3d(smem_u32(v_tile(s)), &vmap, full_bar(s), 0, d.kv, phys * BS, policy);
+      // Each pass, every owner lane whose stage all four consumer warps have
+      // released arms it and issues its two boxes (a non-blocking test, all lanes
+      // in parallel), then fetches the block-table entry of its next stage; when
+      // no lane could issue, one pending lane sleeps on its stage.
+      // The CTA's first item: only two stages go out before the consumers hold
+      // their query fragments, so that the fragment loads are not queued behind
+      // the whole ring's worth of KV requests.
+      bool gated = (done == 0);
+      while (ok) {
+        const bool pending = owner && kk < nst;
+        const unsigned pend = __ballot_sync(kFull, pending);
+        if (pend == 0u) break;
+        bool issued = false;
+        if (pending && !(gated && kk >= 2)) {
+          const int round = (done + kk) / C::kStages;
+          if (round == 0 || mbar_try_wait(empty_bar(lane), (round - 1) & 1)) {
+            const int tok = phys * BS + (kk % C::kSPB) * C::kTok;
+            const int hrow = d.hg * C::kHP;
+            mbar_arrive_expect_tx(full_bar(lane), C::kStageBytes);
+            tma_load_3d(smem_u32(k_tile(lane)), &kmap, full_bar(lane), 0, tok, hrow, policy);
+            tma_load_3d(smem_u32(v_tile(lane)), &vmap, full_bar(lane), 0, tok, hrow, policy);
+            kk += C::kStages;
+            if (kk < nst) phys = load_phys(kk);
+            issued = true;
           }
         }
-        phys_cur = phys_nxt;
-        ok = __all_sync(kFull, mine_ok);
-        if (!ok && lane == 0) record_error(a.err, PA_DEVERR_TIMEOUT);
+        if (__ballot_sync(kFull, issued) == 0u && gated) {
+          if (lane == 0 && !mbar_wait(frag_ready, 0)) {
+            record_error(a.err, PA_DEVERR_TIMEOUT);
+            ok = false;
+          }
+          ok = __shfl_sync(kFull, ok, 0);
+          gated = false;
+        } else if (__ballot_sync(kFull, issued) == 0u) {
+          // nothing was free: sleep on the first pending lane's stage
+          const int l0 = __ffs(pend) - 1;
+          if (lane == l0) {
+            const int round = (done + kk) / C::kStages;
+            if (!mbar_wait(empty_bar(lane), (round - 1) & 1)) {
+              record_error(a.err, PA_DEVERR_TIMEOUT);
+              ok = false;
+            }
+          }
+          ok = __shfl_sync(kFull, ok, l0);
+        }
       }
-      cnt_w0 += warp_blocks<C::kBPI>(d.nloc, 0);
-      cnt_w1 += warp_blocks<C::kBPI>(d.nloc, 1);
-      cnt_w2 += warp_blocks<C::kBPI>(d.nloc, 2);
-      cnt_w3 += warp_blocks<C::kBPI>(d.nloc, 3);
+      done += nst;
       slot ^= 1;
       w = next_index();
     }
     // The last prefetched index is consumed (its atomic has completed) before
     // this CTA signs off.
     const uint32_t last = __shfl_sync(kFull, w_pref, 0);
-    // Leave no copy in flight: wait for the last box of every stage, all within
+    // Leave no copy in flight: wait for the last fill of every stage, all within
     // one bounded window (the consumers normally consumed them already).
     if (lane == 0) {
       const uint64_t deadline = global_timer_ns() + kWaitLimitNs;
       bool fine = true;
-      for (int wq = 0; wq < C::kWarps; ++wq)
-        for (int j = 0; fine && j < C::kSW && j < cnt_of(wq); ++j) {
-          const int last_round = (cnt_of(wq) - 1 - j) / C::kSW;
-          fine = mbar_wait_until(full_bar(wq * C::kSW + j), last_round & 1, deadline);
-        }
+      for (int s = 0; fine && s < C::kStages && s < done; ++s) {
+        const int last_round = (done - 1 - s) / C::kStages;
+        fine = mbar_wait_until(full_bar((done - 1 - s) % C::kStages), last_round & 1, deadline);
+      }
       if (!fine) record_error(a.err, PA_DEVERR_TIMEOUT);
+      if (last == 0xffffffffu) record_error(a.err, PA_DEVERR_BAD_LENGTH);  // (never: uses the value)
       __threadfence();
       // The last CTA to finish rewinds the work counter for the next call.
-      if (last == 0xffffffffu) record_error(a.err, PA_DEVERR_BAD_LENGTH);  // (never: uses the value)
       if (atomicAdd(a.work + 1, 1u) == gridDim.x - 1) {
         a.work[0] = 0u;
         a.work[1] = 0u;
@@ -643,13 +658,12 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
   }
 
   // ======================================================== consumer warps
-  const int tid = threadIdx.x;  // 0..127
   int uses[2] = {0, 0};
   int slot = 0;
-  int kc = 0;  // blocks this warp consumed so far: its k-th block is in stage
-               // warp * kSW + k % kSW of its own sub-ring, round k / kSW
+  bool prep_done = false;  // the fragment pre-pass grid has completed
+  int kc = 0;  // stages consumed so far: item stage it is ring stage (kc + it) % kStages
   // ldmatrix lane addressing: matrix (lane >> 3) covers rows (lane & 7) + 8 * (m & 1)
-  // of a 16-row key tile and chunk (2 cp + (m >> 1)).
+  // of the 16-row head tile and chunk (2 cp + (m >> 1)).
   const int lm = lane >> 3;
   const int ld_row = (lane & 7) + 8 * (lm & 1);
   const int ld_chunk = lm >> 1;
@@ -662,53 +676,68 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
     ++uses[slot];
     const ItemDesc d = descs[slot];
     if (!d.valid) break;
-    const int kv = d.kv, rg = d.rg, b = d.b, split = d.split, q0 = d.q0;
+    const int h = d.hg * C::kHP + warp;  // this warp's KV head
+    const bool active = h < a.Hk;
+    const int split = d.split, q0 = d.q0;
     const int row0 = d.row0, row_end = d.row_end, past = d.past, kmax = d.kmax, kfull = d.kfull;
-    const int blk_begin = d.blk_begin, nloc = d.nloc, nsplit = d.nsplit;
-    const int Lb = d.Lb;
+    const int blk_begin = d.blk_begin, nloc = d.nloc, nsplit = d.nsplit, Lb = d.Lb;
     const int nrows = row_end - row0;
-    const float* sks = reinterpret_cast<const float*>(smem + C::kKsOff) + slot * D;
-    const float* svs = reinterpret_cast<const float*>(smem + C::kVsOff) + slot * D;
+    const int nst = nloc * C::kSPB;
     bool alive = true;
 
-    // ---- prologue: query fragments for this item (cooperative)
-    build_fragments<KV, D, BS, NT, LP>(a, smem + C::kQOff + slot * C::kQBytes, sks, nrows, frag,
-                                       rowc, tid);
-    consumer_sync();
+    // ---- prologue: this head's precomputed query fragments and row multipliers
+    // (written by the pre-pass kernel, which this grid waits for once)
+    const bool first_item = !prep_done;
+    if (!prep_done) {
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      prep_done = true;
+    }
     uint32_t qf[NT][C::kQWords];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int k4 = 0; k4 < C::kQWords / 4; ++k4) {
-        const uint4 v = *reinterpret_cast<const uint4*>(
-            frag + (nt * 32 + lane) * C::kQStride + 4 * k4);
-        qf[nt][4 * k4 + 0] = v.x;
-        qf[nt][4 * k4 + 1] = v.y;
-        qf[nt][4 * k4 + 2] = v.z;
-        qf[nt][4 * k4 + 3] = v.w;
-      }
-    // per accumulator column j: logit weights and causal limit (LP: j = 0 only,
-    // the thread's row is tig)
     float wA[NT][2], wB[NT][2];
     int lim[NT][2];
+    {
+      const uint32_t* fb =
+          a.frag + (static_cast<size_t>(d.b) * a.Hk + (active ? h : 0)) * a.num_row_groups * C::kUnitWords +
+          static_cast<size_t>(d.rg) * C::kUnitWords;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+      for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int rl = LP ? tig : nt * 8 + 2 * tig + j;
-        const float cr = rowc[rl];
-        if constexpr (C::kInt) {
-          const float base = cr * ((KV == PA_KV_INT4) ? (1.f / 131072.f) : (1.f / 8192.f));
-          wA[nt][j] = base;                                            // C 2^-13 (/16 INT4)
-          wB[nt][j] = LP ? base * (1.f / 16384.f) : base * (1.f / 128.f);  // digits 2|3 or 2
-        } else {
-          wA[nt][j] = cr;
-          wB[nt][j] = 0.f;
+        for (int k4 = 0; k4 < C::kQWords / 4; ++k4) {
+          uint4 v = make_uint4(0u, 0u, 0u, 0u);
+          if (active) v = __ldcg(reinterpret_cast<const uint4*>(fb + (nt * 32 + lane) * C::kQWords) + k4);
+          qf[nt][4 * k4 + 0] = v.x;
+          qf[nt][4 * k4 + 1] = v.y;
+          qf[nt][4 * k4 + 2] = v.z;
+          qf[nt][4 * k4 + 3] = v.w;
         }
-        lim[nt][j] = (row0 + rl < row_end && a.causal) ? past + (row0 + rl) / a.G : kmax - 1;
-      }
-    consumer_sync();  // every warp holds its fragments: the area may be reused
+      const float* crow = reinterpret_cast<const float*>(fb + NT * 32 * C::kQWords);
+      // per accumulator column j: logit weights and causal limit (LP: j = 0 only,
+      // the thread's row is tig)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int rl = LP ? tig : nt * 8 + 2 * tig + j;
+          const float cr = active ? __ldcg(crow + rl) : 0.f;
+          if constexpr (C::kInt) {
+            const float base = cr * ((KV == PA_KV_INT4) ? (1.f / 131072.f) : (1.f / 8192.f));
+            wA[nt][j] = base;                                                // C 2^-13 (/16 INT4)
+            wB[nt][j] = LP ? base * (1.f / 16384.f) : base * (1.f / 128.f);  // digits 2|3 or 2
+          } else {
+            wA[nt][j] = cr;
+            wB[nt][j] = 0.f;
+          }
+          lim[nt][j] = (row0 + rl < row_end && a.causal) ? past + (row0 + rl) / a.G : kmax - 1;
+        }
+    }
 
+    if (first_item) {
+      // the fragments are in registers (the empty asm consumes them), then the
+      // producer may release the rest of the first item's stages
+      asm volatile("" ::"r"(qf[0][0]), "r"(qf[0][C::kQWords - 1]), "f"(wA[0][0]), "f"(wA[NT - 1][1]));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(frag_ready);
+    }
     float o[NT][C::kMTiles][4];
     float lacc[NT][4];  // row sums of the fp16 P (ones-matrix MMA)
     float m_run[NT][2], msub[NT][2], thr[NT][2];
@@ -728,39 +757,22 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
       }
     }
 
-    for (int it = warp; alive && it * C::kBPI < nloc; it += C::kWarps) {
-      const int lb0 = it * C::kBPI;
-      const int nb = min(C::kBPI, nloc - lb0);
-      const int ntiles = nb * C::kKeyTiles;
-      for (int bi = 0; bi < nb; ++bi) {
-        // The stage is this warp's own: it consumed round - 1 itself, so the
-        // parity of the wait is unambiguous.
-        const int k = kc + bi;
-        const int s = warp * C::kSW + k % C::kSW, round = k / C::kSW;
-        if (!mbar_wait(full_bar(s), round & 1)) {
-          if (lane == 0) record_error(a.err, PA_DEVERR_TIMEOUT);
-          alive = false;
-        }
+    for (int it = 0; it < nst; ++it) {
+      const int s = (kc + it) % C::kStages, round = (kc + it) / C::kStages;
+      if (alive && !mbar_wait(full_bar(s), round & 1)) {
+        if (lane == 0) record_error(a.err, PA_DEVERR_TIMEOUT);
+        alive = false;
       }
-      if (!alive) break;
-
-      // X: logits in log2 units minus the row's running reference, then P.
-      // LP: X[t][0][eh] = key g + 8 eh of row tig.  Else X[t][nt][e]: key g + 8 (e >> 1),
-      // row nt * 8 + 2 tig + (e & 1).
-      float X[C::kTPI][NT][4];
-#pragma unroll
-      for (int t = 0; t < C::kTPI; ++t) {
-        if (t >= ntiles) {
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) X[t][nt][e] = -INFINITY;
-          continue;
-        }
-        const int bi = t / C::kKeyTiles, kt = t % C::kKeyTiles;
-        const uint32_t kbase = smem_u32(k_tile(warp * C::kSW + (kc + bi) % C::kSW));
-        const int key0 = (blk_begin + lb0 + bi) * BS + kt * 16;
+      if (active && alive) {
+        const uint32_t kbase = smem_u32(k_tile(s) + warp * C::kHeadTile);
+        const uint32_t vbase = smem_u32(v_tile(s) + warp * C::kHeadTile);
+        const int key0 = (blk_begin + it / C::kSPB) * BS + (it % C::kSPB) * C::kTok;
         const bool need_mask = key0 + 16 > kfull;
+
+        // ---------------- QK: X = logits (log2 units) minus the row's reference.
+        // LP: X[0][eh] = key g + 8 eh of row tig.  Else X[nt][e]: key g + 8 (e >> 1),
+        // row nt * 8 + 2 tig + (e & 1).
+        float X[NT][4];
         if constexpr (C::kInt) {
           int acc[C::kAcc][NT][4];
 #pragma unroll
@@ -772,30 +784,30 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
 #pragma unroll
           for (int cp = 0; cp < C::kChunks / 2; ++cp) {
             uint32_t r[4];
-            const uint32_t off = (kt * 16 + ld_row) * C::kCHS + (2 * cp + ld_chunk) * 16;
+            const uint32_t off = ld_row * C::kCHS + (2 * cp + ld_chunk) * 16;
             ldsm_x4(kbase + swz<C::kSwzMask>(off), r);
 #pragma unroll
-            for (int h = 0; h < (KV == PA_KV_INT4 ? 2 : 1); ++h) {
+            for (int hh = 0; hh < (KV == PA_KV_INT4 ? 2 : 1); ++hh) {
               uint32_t a0, a1, a2, a3;
-              int s;
+              int ks;
               if constexpr (KV == PA_KV_INT8) {
                 a0 = r[0]; a1 = r[1]; a2 = r[2]; a3 = r[3];  // 32 channels, raw codes
-                s = cp;
+                ks = cp;
               } else {
                 // nibbles as signed bytes 16 x code: low nibbles shifted up, high masked
-                const uint32_t x0 = r[2 * h], x1 = r[2 * h + 1];  // keys g, g+8; chunk 2cp+h
+                const uint32_t x0 = r[2 * hh], x1 = r[2 * hh + 1];  // keys g, g+8; chunk 2cp+hh
                 a0 = (x0 << 4) & 0xF0F0F0F0u;
                 a1 = (x1 << 4) & 0xF0F0F0F0u;
                 a2 = x0 & 0xF0F0F0F0u;
                 a3 = x1 & 0xF0F0F0F0u;
-                s = 2 * cp + h;
+                ks = 2 * cp + hh;
               }
 #pragma unroll
               for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int i = 0; i < C::kAcc; ++i)
-                  imma_16832<false>(acc[i][nt], a0, a1, a2, a3, qf[nt][(s * C::kAcc + i) * 2],
-                                    qf[nt][(s * C::kAcc + i) * 2 + 1]);
+                  imma_16832<false>(acc[i][nt], a0, a1, a2, a3, qf[nt][(ks * C::kAcc + i) * 2],
+                                    qf[nt][(ks * C::kAcc + i) * 2 + 1]);
             }
           }
           if constexpr (LP) {
@@ -806,7 +818,7 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
               float xv = fmaf(__int2float_rn(A), wA[0][0],
                               fmaf(__int2float_rn(B2), wB[0][0], -msub[0][0]));
               if (need_mask && key0 + g + 8 * eh > lim[0][0]) xv = -INFINITY;
-              X[t][0][eh] = xv;
+              X[0][eh] = xv;
             }
           } else {
 #pragma unroll
@@ -818,7 +830,7 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
                 float xv = fmaf(__int2float_rn(A), wA[nt][j],
                                 fmaf(__int2float_rn(acc[2][nt][e]), wB[nt][j], -msub[nt][j]));
                 if (need_mask && key0 + g + (e >> 1) * 8 > lim[nt][j]) xv = -INFINITY;
-                X[t][nt][e] = xv;
+                X[nt][e] = xv;
               }
           }
         } else {
@@ -832,20 +844,20 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
 #pragma unroll
           for (int cp = 0; cp < C::kChunks / 2; ++cp) {
             uint32_t r[4];
-            const uint32_t off = (kt * 16 + ld_row) * C::kCHS + (2 * cp + ld_chunk) * 16;
+            const uint32_t off = ld_row * C::kCHS + (2 * cp + ld_chunk) * 16;
             ldsm_x4(kbase + swz<C::kSwzMask>(off), r);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int s = 2 * cp + h;  // 16-channel k-step
+            for (int hh = 0; hh < 2; ++hh) {
+              const int ks = 2 * cp + hh;  // 16-channel k-step
               uint32_t a0, a1, a2, a3;
-              e4m3x4_to_h2x2(r[2 * h], a0, a2);      // key g: channels +0,1 | +2,3
-              e4m3x4_to_h2x2(r[2 * h + 1], a1, a3);  // key g+8
+              e4m3x4_to_h2x2(r[2 * hh], a0, a2);      // key g: channels +0,1 | +2,3
+              e4m3x4_to_h2x2(r[2 * hh + 1], a1, a3);  // key g+8
 #pragma unroll
               for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int i = 0; i < C::kAcc; ++i)
-                  mma_16816(sacc[i][nt], a0, a1, a2, a3, qf[nt][(s * C::kAcc + i) * 2],
-                            qf[nt][(s * C::kAcc + i) * 2 + 1]);
+                  mma_16816(sacc[i][nt], a0, a1, a2, a3, qf[nt][(ks * C::kAcc + i) * 2],
+                            qf[nt][(ks * C::kAcc + i) * 2 + 1]);
             }
           }
           if constexpr (LP) {
@@ -854,7 +866,7 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
               // columns 2 tig / 2 tig + 1: high part / residual of row tig
               float xv = fmaf(sacc[0][0][2 * eh] + sacc[0][0][2 * eh + 1], wA[0][0], -msub[0][0]);
               if (need_mask && key0 + g + 8 * eh > lim[0][0]) xv = -INFINITY;
-              X[t][0][eh] = xv;
+              X[0][eh] = xv;
             }
           } else {
 #pragma unroll
@@ -864,105 +876,88 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
                 const int j = e & 1;
                 float xv = fmaf(sacc[0][nt][e] + sacc[1][nt][e], wA[nt][j], -msub[nt][j]);
                 if (need_mask && key0 + g + (e >> 1) * 8 > lim[nt][j]) xv = -INFINITY;
-                X[t][nt][e] = xv;
+                X[nt][e] = xv;
               }
           }
         }
-      }
 
-      // ---------------- online softmax with a lazily raised running max
-      if constexpr (LP) {
-        float mx = fmaxf(fmaxf(X[0][0][0], X[0][0][1]), fmaxf(X[1][0][0], X[1][0][1]));
-        if (__any_sync(kFull, mx > thr[0][0])) {
-          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
-          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
-          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
-          if (mx > thr[0][0]) {
-            const float mnew = mx + msub[0][0];
-            const float alpha = (m_run[0][0] == -INFINITY) ? 0.f : fast_exp2(m_run[0][0] - mnew);
+        // ---------------- online softmax with a lazily raised running max
+        if constexpr (LP) {
+          float mx = fmaxf(X[0][0], X[0][1]);
+          if (__any_sync(kFull, mx > thr[0][0])) {
+            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
+            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
+            if (mx > thr[0][0]) {
+              const float mnew = mx + msub[0][0];
+              const float alpha =
+                  (m_run[0][0] == -INFINITY) ? 0.f : fast_exp2(m_run[0][0] - mnew);
 #pragma unroll
-            for (int mt = 0; mt < C::kMTiles; ++mt)
+              for (int mt = 0; mt < C::kMTiles; ++mt)
 #pragma unroll
-              for (int e = 0; e < 4; ++e) o[0][mt][e] *= alpha;
+                for (int e = 0; e < 4; ++e) o[0][mt][e] *= alpha;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) lacc[0][e] *= alpha;
-#pragma unroll
-            for (int t = 0; t < C::kTPI; ++t) {
-              X[t][0][0] -= mx;
-              X[t][0][1] -= mx;
+              for (int e = 0; e < 4; ++e) lacc[0][e] *= alpha;
+              X[0][0] -= mx;
+              X[0][1] -= mx;
+              m_run[0][0] = mnew;
+              msub[0][0] = mnew;
+              thr[0][0] = 8.f;
             }
-            m_run[0][0] = mnew;
-            msub[0][0] = mnew;
-            thr[0][0] = 8.f;
           }
-        }
-#pragma unroll
-        for (int t = 0; t < C::kTPI; ++t) {
-          X[t][0][0] = fast_exp2(X[t][0][0]);  // <= 2^8: safe range for fp16
-          X[t][0][1] = fast_exp2(X[t][0][1]);
-        }
-      } else {
-        float mx[NT][2];
-        bool any = false;
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            mx[nt][j] = fmaxf(fmaxf(X[0][nt][j], X[0][nt][j + 2]),
-                              fmaxf(X[1][nt][j], X[1][nt][j + 2]));
-            any |= mx[nt][j] > thr[nt][j];
-          }
-        if (__any_sync(kFull, any)) {
+          X[0][0] = fast_exp2(X[0][0]);  // <= 2^8: safe range for fp16
+          X[0][1] = fast_exp2(X[0][1]);
+        } else {
+          float mx[NT][2];
+          bool any = false;
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-              float m = mx[nt][j];
-              m = fmaxf(m, __shfl_xor_sync(kFull, m, 4));
-              m = fmaxf(m, __shfl_xor_sync(kFull, m, 8));
-              m = fmaxf(m, __shfl_xor_sync(kFull, m, 16));
-              if (m > thr[nt][j]) {
-                const float mnew = m + msub[nt][j];
-                const float alpha =
-                    (m_run[nt][j] == -INFINITY) ? 0.f : fast_exp2(m_run[nt][j] - mnew);
-#pragma unroll
-                for (int mt = 0; mt < C::kMTiles; ++mt) {
-                  o[nt][mt][j] *= alpha;
-                  o[nt][mt][j + 2] *= alpha;
-                }
-                lacc[nt][j] *= alpha;
-                lacc[nt][j + 2] *= alpha;
-#pragma unroll
-                for (int t = 0; t < C::kTPI; ++t) {
-                  X[t][nt][j] -= m;
-                  X[t][nt][j + 2] -= m;
-                }
-                m_run[nt][j] = mnew;
-                msub[nt][j] = mnew;
-                thr[nt][j] = 8.f;
-              }
+              mx[nt][j] = fmaxf(X[nt][j], X[nt][j + 2]);
+              any |= mx[nt][j] > thr[nt][j];
             }
-        }
+          if (__any_sync(kFull, any)) {
 #pragma unroll
-        for (int t = 0; t < C::kTPI; ++t)
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+              for (int j = 0; j < 2; ++j) {
+                float m = mx[nt][j];
+                m = fmaxf(m, __shfl_xor_sync(kFull, m, 4));
+                m = fmaxf(m, __shfl_xor_sync(kFull, m, 8));
+                m = fmaxf(m, __shfl_xor_sync(kFull, m, 16));
+                if (m > thr[nt][j]) {
+                  const float mnew = m + msub[nt][j];
+                  const float alpha =
+                      (m_run[nt][j] == -INFINITY) ? 0.f : fast_exp2(m_run[nt][j] - mnew);
+#pragma unroll
+                  for (int mt = 0; mt < C::kMTiles; ++mt) {
+                    o[nt][mt][j] *= alpha;
+                    o[nt][mt][j + 2] *= alpha;
+                  }
+                  lacc[nt][j] *= alpha;
+                  lacc[nt][j + 2] *= alpha;
+                  X[nt][j] -= m;
+                  X[nt][j + 2] -= m;
+                  m_run[nt][j] = mnew;
+                  msub[nt][j] = mnew;
+                  thr[nt][j] = 8.f;
+                }
+              }
+          }
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) X[t][nt][e] = fast_exp2(X[t][nt][e]);
-      }
+            for (int e = 0; e < 4; ++e) X[nt][e] = fast_exp2(X[nt][e]);
+        }
 
-      // ---------------- O^T[dim, col] += V^T P^T, per key tile
-#pragma unroll
-      for (int t = 0; t < C::kTPI; ++t) {
-        if (t >= ntiles) continue;
-        const int bi = t / C::kKeyTiles, kt = t % C::kKeyTiles;
-        const uint32_t vbase = smem_u32(v_tile(warp * C::kSW + (kc + bi) % C::kSW));
+        // ---------------- O^T[dim, col] += V^T P^T
         uint32_t pb[NT][2];
         if constexpr (LP) {
           // (row tig; keys g, g+8) -> column n = g: b0 (keys 2tig, 2tig+1) and b1
           // (keys 2tig+8, 2tig+9) of row n / 2; movmatrix gives even lanes b0 and
           // odd lanes b1, the partner lane (lane ^ 4) the other.
-          const uint32_t p = pack_f32x2_to_h2(X[t][0][0], X[t][0][1]);
+          const uint32_t p = pack_f32x2_to_h2(X[0][0], X[0][1]);
           const uint32_t mtr = movmatrix_trans(p);
           const uint32_t y = __shfl_xor_sync(kFull, mtr, 4);
           pb[0][0] = (g & 1) ? y : mtr;
@@ -970,23 +965,22 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
         } else {
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
-            pb[nt][0] = movmatrix_trans(pack_f32x2_to_h2(X[t][nt][0], X[t][nt][1]));
-            pb[nt][1] = movmatrix_trans(pack_f32x2_to_h2(X[t][nt][2], X[t][nt][3]));
+            pb[nt][0] = movmatrix_trans(pack_f32x2_to_h2(X[nt][0], X[nt][1]));
+            pb[nt][1] = movmatrix_trans(pack_f32x2_to_h2(X[nt][2], X[nt][3]));
           }
         }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
           mma_16816(lacc[nt], kOnesH2, kOnesH2, kOnesH2, kOnesH2, pb[nt][0], pb[nt][1]);
-        const int tkey0 = (blk_begin + lb0 + bi) * BS + kt * 16;
 #pragma unroll
         for (int cp = 0; cp < C::kChunks / 2; ++cp) {
           uint32_t r[4];
-          const uint32_t off = (kt * 16 + ld_row) * C::kCHS + (2 * cp + ld_chunk) * 16;
+          const uint32_t off = ld_row * C::kCHS + (2 * cp + ld_chunk) * 16;
           ldsm_x4_trans(vbase + swz<C::kSwzMask>(off), r);
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t lo = r[2 * h], hi = r[2 * h + 1];  // keys 2tig.. / 2tig+8.. of chunk c
-            const int c = 2 * cp + h;
+          for (int hf = 0; hf < 2; ++hf) {
+            const uint32_t lo = r[2 * hf], hi = r[2 * hf + 1];  // keys 2tig.. / 2tig+8.. of chunk c
+            const int c = 2 * cp + hf;
 #pragma unroll
             for (int hh = 0; hh < (KV == PA_KV_INT4 ? 2 : 1); ++hh) {
               uint32_t a0, a1, a2, a3;
@@ -1002,10 +996,10 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
               } else if constexpr (KV == PA_KV_FP8_E4M3) {
                 e4m3x4_to_h2x2(prmt(lo, 0u, 0x3120), a0, a1);
                 e4m3x4_to_h2x2(prmt(hi, 0u, 0x3120), a2, a3);
-                if (tkey0 + 16 > Lb) {
+                if (key0 + 16 > Lb) {
                   // Keys past the sequence end hold stale bytes; an FP8 NaN there would
                   // poison P*V even with P = 0, so such V codes are zeroed.
-                  const int kb = tkey0 + 2 * tig;
+                  const int kb = key0 + 2 * tig;
                   const uint32_t mlo = (kb < Lb ? 0x0000ffffu : 0u) | (kb + 1 < Lb ? 0xffff0000u : 0u);
                   const uint32_t mhi =
                       (kb + 8 < Lb ? 0x0000ffffu : 0u) | (kb + 9 < Lb ? 0xffff0000u : 0u);
@@ -1032,94 +1026,32 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
         }
       }
       __syncwarp();
-      if (lane == 0)
-        for (int bi = 0; bi < nb; ++bi) mbar_arrive(empty_bar(warp * C::kSW + (kc + bi) % C::kSW));
-      kc += nb;
+      if (lane == 0) mbar_arrive(empty_bar(s));
     }
+    kc += nst;
 
-    // ---- this warp's result: remove the code->fp16 constants (using the exact
-    // row sums of P); columns j of the accumulators (LP: both = row tig)
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int mt = 0; mt < C::kMTiles; ++mt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float l = lacc[nt][LP ? 0 : (e & 1)];
-          if constexpr (KV == PA_KV_INT8) {
-            o[nt][mt][e] = fmaf(-1152.f, l, o[nt][mt][e]);
-          } else if constexpr (KV == PA_KV_INT4) {
-            o[nt][mt][e] = (e < 2) ? fmaf(-1032.f, l, o[nt][mt][e])
-                                   : fmaf(-1152.f, l, o[nt][mt][e]) * (1.f / 16.f);
-          }
-        }
-
-    // ---- merge the four warps' (m, l, O); warp 0 ends with the total.
-    // Slice rows are [row][D] fp32 with swizzled dim pairs.
-    auto slice_sw = [&](int row) { return LP ? (row & 3) : ((row >> 1) & 3); };
-    auto write_slice = [&](float* sl, float* ml) {
+    if (active && alive) {
+      // ---- remove the code->fp16 constants (using the exact row sums of P);
+      // accumulator columns j (LP: both = row tig)
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int j = 0; j < (LP ? 1 : 2); ++j) {
-          const int row = LP ? tig : nt * 8 + 2 * tig + j;
+        for (int mt = 0; mt < C::kMTiles; ++mt)
 #pragma unroll
-          for (int mt = 0; mt < C::kMTiles; ++mt) {
-            const int dcol = slice_col(out_dim<KV>(mt, g), slice_sw(row));
-            *reinterpret_cast<float2*>(sl + row * D + dcol) =
-                make_float2(o[nt][mt][j], o[nt][mt][j + 2]);
+          for (int e = 0; e < 4; ++e) {
+            const float l = lacc[nt][LP ? 0 : (e & 1)];
+            if constexpr (KV == PA_KV_INT8) {
+              o[nt][mt][e] = fmaf(-1152.f, l, o[nt][mt][e]);
+            } else if constexpr (KV == PA_KV_INT4) {
+              o[nt][mt][e] = (e < 2) ? fmaf(-1032.f, l, o[nt][mt][e])
+                                     : fmaf(-1152.f, l, o[nt][mt][e]) * (1.f / 16.f);
+            }
           }
-          if (g == 0) {
-            ml[row] = m_run[nt][j];
-            ml[C::kRows + row] = lacc[nt][LP ? 0 : j];
-          }
-        }
-    };
-    // Adds a slice (m_s, l_s, O_s) into this warp's (m, l, O).
-    auto merge_slice = [&](const float* sl, const float* ml) {
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int j = 0; j < (LP ? 1 : 2); ++j) {
-          const int row = LP ? tig : nt * 8 + 2 * tig + j;
-          const float ms = ml[row], ls = ml[C::kRows + row];
-          const float M = fmaxf(m_run[nt][j], ms);
-          const float fo = (m_run[nt][j] == -INFINITY) ? 0.f : fast_exp2(m_run[nt][j] - M);
-          const float fs = (ms == -INFINITY) ? 0.f : fast_exp2(ms - M);
-#pragma unroll
-          for (int mt = 0; mt < C::kMTiles; ++mt) {
-            const int dcol = slice_col(out_dim<KV>(mt, g), slice_sw(row));
-            const float2 v = *reinterpret_cast<const float2*>(sl + row * D + dcol);
-            o[nt][mt][j] = fmaf(v.x, fs, o[nt][mt][j] * fo);
-            o[nt][mt][j + 2] = fmaf(v.y, fs, o[nt][mt][j + 2] * fo);
-          }
-          const int jl = LP ? 0 : j;
-          lacc[nt][jl] = fmaf(ls, fs, lacc[nt][jl] * fo);
-          m_run[nt][j] = M;
-        }
-    };
-    if constexpr (LP) {
-      if (warp > 0) write_slice(slices + (warp - 1) * C::kSliceBytes / 4,
-                                sm_ml + (warp - 1) * 2 * C::kRows);
-      consumer_sync();
-      if (warp == 0)
-#pragma unroll
-        for (int sl = 0; sl < C::kSlices; ++sl)
-          merge_slice(slices + sl * C::kSliceBytes / 4, sm_ml + sl * 2 * C::kRows);
-      consumer_sync();
-    } else {
-      for (int wsum = C::kWarps - 1; wsum >= 0; --wsum) {
-        if (warp == wsum) {
-          if (wsum != C::kWarps - 1) merge_slice(slices, sm_ml);
-          if (wsum != 0) write_slice(slices, sm_ml);
-        }
-        consumer_sync();
-      }
-    }
 
-    // ---- warp 0: normalise, apply the V scale, store the output or the split partial
-    if (warp == 0) {
+      // ---- normalise, apply the V scale, store the rows or the split partial
       const bool is_split = nsplit > 1;
+      const float* vsc = a.v_scale + static_cast<size_t>(h) * D;
+      const size_t stride = static_cast<size_t>(a.total_q) * a.H;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -1127,14 +1059,14 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
           const int rl = LP ? tig : nt * 8 + 2 * tig + j;
           if (rl >= nrows) continue;
           const int r = row0 + rl;
-          const size_t orow = static_cast<size_t>(q0 + r / a.G) * a.H + kv * a.G + r % a.G;
+          const size_t orow = static_cast<size_t>(q0 + r / a.G) * a.H + h * a.G + r % a.G;
           const float L = lacc[nt][LP ? 0 : j];
           const float inv = (L > 0.f) ? 1.f / L : 0.f;
-          const size_t prow = static_cast<size_t>(split) * a.total_q * a.H + orow;
+          const size_t prow = static_cast<size_t>(split) * stride + orow;
 #pragma unroll
           for (int mt = 0; mt < C::kMTiles; ++mt) {
             const int dd = out_dim<KV>(mt, g);
-            const float2 vs = *reinterpret_cast<const float2*>(svs + dd);
+            const float2 vs = __ldg(reinterpret_cast<const float2*>(vsc + dd));
             const float o0 = o[nt][mt][j] * inv * vs.x;
             const float o1 = o[nt][mt][j + 2] * inv * vs.y;
             if (!is_split) {
@@ -1151,105 +1083,134 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
           if (is_split && g == 0)
             a.lse_part[prow] = (L > 0.f) ? m_run[nt][j] + __log2f(L) : -INFINITY;
         }
-      if (is_split) {
-        // publish this split and count arrivals; the last split of the unit
-        // merges all of them and rewinds the counter for the next call
-        __threadfence();
-        __syncwarp();
-        uint32_t* counter =
-            a.counters + (static_cast<size_t>(b) * a.Hk + kv) * a.num_row_groups + rg;
-        int last = 0;
-        if (lane == 0) last = (atomicAdd(counter, 1u) == static_cast<uint32_t>(nsplit - 1));
-        last = __shfl_sync(kFull, last, 0);
-        if (lane == 0) *sm_flag = last;
-      }
-      if (lane == 0 && !is_split) *sm_flag = 0;
+
     }
-    if (nsplit > 1) {
-      consumer_sync();
-      if (*sm_flag) {
-        __threadfence();
-        const size_t stride = static_cast<size_t>(a.total_q) * a.H;
-        const int S = nsplit;
-        const int nthr = C::kWarps * 32;
-        // 1) every (split, row) log2-sum-exp
-        for (int idx = tid; idx < S * nrows; idx += nthr) {
-          const int s = idx / nrows, row = idx % nrows;
-          const int r = row0 + row;
-          const size_t orow = static_cast<size_t>(q0 + r / a.G) * a.H + kv * a.G + r % a.G;
-          wts[s * C::kRows + row] = __ldcg(a.lse_part + s * stride + orow);
-        }
-        consumer_sync();
-        // 2) per row (one warp per row): weights 2^(lse_s - max) / sum
-        for (int row = warp; row < nrows; row += C::kWarps) {
-          float M = -INFINITY;
-          for (int s = lane; s < S; s += 32) M = fmaxf(M, wts[s * C::kRows + row]);
-#pragma unroll
-          for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o2));
-          float sum = 0.f;
-          for (int s = lane; s < S; s += 32) {
-            const float ls = wts[s * C::kRows + row];
-            const float wgt = (ls == -INFINITY) ? 0.f : fast_exp2(ls - M);
-            wts[s * C::kRows + row] = wgt;
-            sum += wgt;
-          }
-#pragma unroll
-          for (int o2 = 16; o2 > 0; o2 >>= 1) sum += __shfl_xor_sync(kFull, sum, o2);
-          const float inv = sum > 0.f ? 1.f / sum : 0.f;
-          __syncwarp();
-          for (int s = lane; s < S; s += 32) wts[s * C::kRows + row] *= inv;
-        }
-        consumer_sync();
-        // 3) weighted sum of the partials, eight splits in flight per thread
-        for (int idx = tid; idx < nrows * (D / 4); idx += nthr) {
-          const int row = idx / (D / 4);
-          const int dd = (idx % (D / 4)) * 4;
-          const int r = row0 + row;
-          const size_t orow = static_cast<size_t>(q0 + r / a.G) * a.H + kv * a.G + r % a.G;
-          const float* base = a.o_part + orow * D + dd;
-          float4 acc4 = make_float4(0.f, 0.f, 0.f, 0.f);
-          for (int s8 = 0; s8 < S; s8 += 8) {
-            float4 v[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-              v[u] = (s8 + u < S)
-                         ? __ldcg(reinterpret_cast<const float4*>(base + (s8 + u) * stride * D))
-                         : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              if (s8 + u < S) {
-                const float wgt = wts[(s8 + u) * C::kRows + row];
-                acc4.x = fmaf(wgt, v[u].x, acc4.x);
-                acc4.y = fmaf(wgt, v[u].y, acc4.y);
-                acc4.z = fmaf(wgt, v[u].z, acc4.z);
-                acc4.w = fmaf(wgt, v[u].w, acc4.w);
-              }
-            }
-          }
-          if (a.out_bf16) {
-            __nv_bfloat162* dst =
-                reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(a.out) +
-                                                  orow * D + dd);
-            dst[0] = __floats2bfloat162_rn(acc4.x, acc4.y);
-            dst[1] = __floats2bfloat162_rn(acc4.z, acc4.w);
-          } else {
-            __half2* dst = reinterpret_cast<__half2*>(reinterpret_cast<__half*>(a.out) + orow * D + dd);
-            dst[0] = __floats2half2_rn(acc4.x, acc4.y);
-            dst[1] = __floats2half2_rn(acc4.z, acc4.w);
-          }
-        }
-        if (tid == 0)
-          a.counters[(static_cast<size_t>(b) * a.Hk + kv) * a.num_row_groups + rg] = 0u;
-      }
-      consumer_sync();  // weights / flag consumed before the next item's prologue
-    }
-    // the item slot (query rows, scales, descriptor) may be refilled
-    if (warp == 0) {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(item_empty(slot));
-    }
+    // the descriptor slot may be refilled
+    __syncwarp();
+    if (lane == 0) mbar_arrive(item_empty(slot));
     slot ^= 1;
   }
+}
+
+// ---------------------------------------------------------------------------
+// Log-sum-exp merge of the split partials (flash decoding, GQA GEMV decode page,
+// Code analysis 2: the workers' partials are combined after the split pass):
+//   lse = log2 sum_s 2^lse_s,  out = sum_s 2^(lse_s - lse) o_s
+// One warp per (new-token row, query head).  The warp recomputes, from the device
+// lengths and the plan, how many splits of its (sequence, KV head, row group)
+// have keys, exactly as the forward kernel decoded its items; rows of unsplit
+// units were stored by the forward kernel and are skipped.  Launched as the
+// forward kernel's programmatic dependent: it waits for the forward grid to
+// complete before reading a partial.
+template <int D, int BS>
+__global__ void __launch_bounds__(128) pa_combine_kernel(const FwdArgs a) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int lane = threadIdx.x & 31;
+  const int gr = blockIdx.x * 4 + (threadIdx.x >> 5);  // row of out viewed as [total_q * H]
+  if (gr >= a.total_q * a.H) return;
+  const int qrow = gr / a.H, hq = gr % a.H;
+  // sequence of the token: the last b with cu[b] <= qrow
+  int lo = 0, hi = a.batch - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(a.cu_seqlens_q + mid) <= qrow) lo = mid; else hi = mid - 1;
+  }
+  const int b = lo;
+  const int q0 = __ldg(a.cu_seqlens_q + b), qb = __ldg(a.cu_seqlens_q + b + 1) - q0;
+  const int Lb = __ldg(a.seqlens_k + b);
+  if (qb <= 0 || qb > Lb) return;
+  const int R = qb * a.G;
+  const int r = (qrow - q0) * a.G + hq % a.G;  // row within the (sequence, KV head) unit
+  const int row0 = (r / a.rows_cta) * a.rows_cta;
+  const int row_end = min(R, row0 + a.rows_cta);
+  const int i_last = (row_end - 1) / a.G;
+  const int kmax = a.causal ? (Lb - qb) + i_last + 1 : Lb;
+  int ns, bps;
+  split_geometry((Lb + BS - 1) / BS, a.split_target, a.max_splits, &ns, &bps);
+  const int S = ((kmax + BS - 1) / BS + bps - 1) / bps;
+  if (S <= 1) return;
+  const size_t stride = static_cast<size_t>(a.total_q) * a.H;
+  // weights 2^(lse_s - max) / sum; lane holds splits lane, lane + 32, ...
+  float ls[4];
+  float M = -INFINITY;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int sp = lane + 32 * k;
+    ls[k] = sp < S ? __ldcg(a.lse_part + sp * stride + gr) : -INFINITY;
+    M = fmaxf(M, ls[k]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
+  float sum = 0.f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    ls[k] = (ls[k] == -INFINITY) ? 0.f : fast_exp2(ls[k] - M);
+    sum += ls[k];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(kFull, sum, o);
+  const float inv = sum > 0.f ? 1.f / sum : 0.f;
+  // lane handles dims 4 lane .. 4 lane + 3
+  constexpr int kD4 = D / 4;
+  const bool dl = lane < kD4;
+  const float* base = a.o_part + static_cast<size_t>(gr) * D + 4 * (dl ? lane : 0);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s8 = 0; s8 < S; s8 += 8) {
+    float4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      v[u] = (s8 + u < S && dl)
+                 ? __ldcg(reinterpret_cast<const float4*>(base + (s8 + u) * stride * D))
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int sp = s8 + u;
+      const float wv = __shfl_sync(kFull, ls[(sp >> 5) & 3], sp & 31) * inv;
+      if (sp < S) {
+        acc.x = fmaf(wv, v[u].x, acc.x);
+        acc.y = fmaf(wv, v[u].y, acc.y);
+        acc.z = fmaf(wv, v[u].z, acc.z);
+        acc.w = fmaf(wv, v[u].w, acc.w);
+      }
+    }
+  }
+  if (dl) {
+    const size_t o = static_cast<size_t>(gr) * D + 4 * lane;
+    if (a.out_bf16) {
+      __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(a.out) + o);
+      dst[0] = __floats2bfloat162_rn(acc.x, acc.y);
+      dst[1] = __floats2bfloat162_rn(acc.z, acc.w);
+    } else {
+      __half2* dst = reinterpret_cast<__half2*>(reinterpret_cast<__half*>(a.out) + o);
+      dst[0] = __floats2half2_rn(acc.x, acc.y);
+      dst[1] = __floats2half2_rn(acc.z, acc.w);
+    }
+  }
+}
+
+template <int D, int BS>
+static cudaError_t launch_combine_t(const FwdArgs& a, cudaStream_t stream) {
+  const long long rows = static_cast<long long>(a.total_q) * a.H;
+  if (rows <= 0) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((rows + 3) / 4));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, pa_combine_kernel<D, BS>, a);
+}
+
+cudaError_t launch_combine(int head_size, int block_size, const FwdArgs& a, cudaStream_t stream) {
+  if (head_size == 64 && block_size == 16) return launch_combine_t<64, 16>(a, stream);
+  if (head_size == 64 && block_size == 32) return launch_combine_t<64, 32>(a, stream);
+  if (head_size == 128 && block_size == 16) return launch_combine_t<128, 16>(a, stream);
+  if (head_size == 128 && block_size == 32) return launch_combine_t<128, 32>(a, stream);
+  return cudaErrorInvalidValue;
 }
 
 template <int KV, int D, int BS, int NT, bool LP>
@@ -1266,6 +1227,19 @@ static cudaError_t launch_t(const CUtensorMap& kmap, const CUtensorMap& vmap, Fw
   if (per_sm == 0) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
+    // All three kernels of a call prefer the largest shared-memory carveout, so
+    // an SM that ran a pre-pass or combine CTA need not be reconfigured before
+    // it can take forward CTAs.
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(pa_prep_kernel<KV, D, BS, NT, LP>,
+                             cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(pa_combine_kernel<D, BS>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, C::kThreads, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
@@ -1274,13 +1248,52 @@ static cudaError_t launch_t(const CUtensorMap& kmap, const CUtensorMap& vmap, Fw
   const long long slots = static_cast<long long>(per_sm) * a.num_sms;
   const int grid = static_cast<int>(a.num_items < slots ? a.num_items : slots);
   if (grid < 1) return cudaSuccess;
-  kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(kmap, vmap, a);
-  return cudaGetLastError();
+  // the fragment pre-pass, then the forward kernel as its programmatic dependent
+  const long long units = static_cast<long long>(a.batch) * a.Hk * a.num_row_groups;
+  pa_prep_kernel<KV, D, BS, NT, LP><<<static_cast<unsigned>((units + 1) / 2), 64, 0, stream>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, kmap, vmap, a);
 }
 
 template <int KV, int D, int BS, int NT, bool LP>
 static int smem_t() {
   return Cfg<KV, D, BS, NT, LP>::kSmemBytes;
+}
+
+template <int KV, int D>
+static int unit_words_t(int rows) {
+  if (rows == 4) return Cfg<KV, D, 16, 1, true>::kUnitWords;
+  if (rows == 8) return Cfg<KV, D, 16, 1, false>::kUnitWords;
+  if (rows == 16) return Cfg<KV, D, 16, 2, false>::kUnitWords;
+  return -1;
+}
+
+int fragment_unit_words(int kv_dtype, int head_size, int rows_per_cta) {
+  const bool d128 = head_size == 128;
+  switch (kv_dtype) {
+    case PA_KV_INT8:
+      return d128 ? unit_words_t<PA_KV_INT8, 128>(rows_per_cta)
+                  : unit_words_t<PA_KV_INT8, 64>(rows_per_cta);
+    case PA_KV_INT4:
+      return d128 ? unit_words_t<PA_KV_INT4, 128>(rows_per_cta)
+                  : unit_words_t<PA_KV_INT4, 64>(rows_per_cta);
+    case PA_KV_FP8_E4M3:
+      return d128 ? unit_words_t<PA_KV_FP8_E4M3, 128>(rows_per_cta)
+                  : unit_words_t<PA_KV_FP8_E4M3, 64>(rows_per_cta);
+    default:
+      return -1;
+  }
 }
 
 int forward_ctas_per_sm(int kv_dtype, int head_size, int block_size, int rows_per_cta) {

@@ -20,11 +20,12 @@ struct FwdArgs {
   const int32_t* cu_seqlens_q;
   float* o_part;        // [max_splits, total_q * H, D] (split mode only)
   float* lse_part;      // [max_splits, total_q * H] (log2 domain)
-  uint32_t* counters;   // [batch * Hk * num_row_groups] split arrival counters (self-resetting)
+  uint32_t* frag;       // [batch * Hk * num_row_groups] precomputed query fragment units
   uint32_t* work;       // [2]: next work item, CTAs finished (both rewound by the last CTA)
   uint32_t* err;        // sticky device error word
   int batch, H, Hk, G, maxb, num_blocks, total_q;
   int q_bf16, out_bf16, causal;
+  int rows_cta;         // query rows per (KV head, row group): 4, 8 or 16
   int num_row_groups;   // largest number of row groups of a (sequence, KV head)
   int max_splits;       // partial slots: no sequence is split into more items
   int split_target;     // KV blocks per split target T: n blocks -> min(max_splits, ceil(n / T))
@@ -33,6 +34,10 @@ struct FwdArgs {
   int num_sms;          // SMs of the device
   float sm_scale_log2;  // softmax_scale * log2(e)
 };
+
+// KV heads of one work item: the fused kernel streams their rows of a block with
+// one TMA box and gives each to one consumer warp.
+constexpr int kHeadsPerItem = 4;
 
 // Split geometry of a sequence with nblk KV blocks for split target T: the
 // number of non-empty splits and the blocks per split.  Shared by the planner
@@ -48,8 +53,8 @@ __host__ __device__ inline void split_geometry(int nblk, int T, int max_splits, 
 }
 
 // Workspace layout: [0, 256) header: error word at byte 0, work counters at
-// byte 64; then the split counters; then the partial outputs and their
-// log-sum-exps (256-byte aligned each).
+// byte 64; then the precomputed query fragments; then the split partial outputs
+// and their log-sum-exps (256-byte aligned each).
 constexpr size_t kWsHeaderBytes = 256;
 constexpr size_t kWsWorkOffset = 64;
 
@@ -58,8 +63,13 @@ constexpr size_t kWsWorkOffset = 64;
 cudaError_t launch_forward(int kv_dtype, int head_size, int block_size, int rows_per_cta,
                            const CUtensorMap& kmap, const CUtensorMap& vmap, const FwdArgs& a,
                            cudaStream_t stream);
+// Log-sum-exp merge of the split partials (one warp per row of a split unit),
+// launched right after the forward kernel as its programmatic dependent.
+cudaError_t launch_combine(int head_size, int block_size, const FwdArgs& a, cudaStream_t stream);
 // Dynamic shared memory of one forward CTA (-1 for an unsupported combination).
 int forward_smem_bytes(int kv_dtype, int head_size, int block_size, int rows_per_cta);
+// 32-bit words of one precomputed query-fragment unit (sequence, KV head, row group).
+int fragment_unit_words(int kv_dtype, int head_size, int rows_per_cta);
 // Forward CTAs resident per SM, from the launch bounds and shared memory.
 int forward_ctas_per_sm(int kv_dtype, int head_size, int block_size, int rows_per_cta);
 

@@ -90,15 +90,9 @@ pa_status paged_attn_forward_noalloc(const void* q, const void* k_cache, const v
   if (st != PA_OK) return st;
 
   // The array keeps the previous call's contents.  Zero what the kernel expects
-  // to start at zero: the error word and work counters (the header) and, when
-  // the plan splits the KV, the per-unit arrival counters behind it.  The split
-  // partials are always written before they are read.
+  // to start at zero: the error word and the work counters (the header).  The
+  // split partials are always written before they are read.
   size_t clear = pa::kWsHeaderBytes;
-  if (params->num_splits > 1) {
-    const size_t units = static_cast<size_t>(params->batch) * params->kv_num_heads *
-                         static_cast<size_t>(params->num_row_groups);
-    clear += units * sizeof(uint32_t);
-  }
   if (clear > need) clear = need;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(scratch, 0, clear, s);

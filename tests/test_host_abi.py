@@ -70,7 +70,7 @@ def test_plan_zero_new_tokens_everywhere_is_a_no_op():
 def _count_items(cu, L, G, Hk, bs, rows, T, max_splits):
     """Work items by the documented split rule: a sequence with n KV blocks gets
     s = min(max_splits, ceil(n / T)) splits of ceil(n / s) blocks (empty ones
-    dropped), times Hk KV heads times its row groups."""
+    dropped), times its groups of 4 KV heads times its row groups."""
     total, most = 0, 1
     for b in range(len(L)):
         qb = int(cu[b + 1] - cu[b])
@@ -81,7 +81,7 @@ def _count_items(cu, L, G, Hk, bs, rows, T, max_splits):
         per = -(-n // s)
         s = -(-n // per)
         most = max(most, s)
-        total += Hk * (-(-qb * G // rows)) * s
+        total += (-(-Hk // 4)) * (-(-qb * G // rows)) * s
     return total, most
 
 
