@@ -61,7 +61,7 @@ WsLayout ws_layout(const paged_attn_params* p) {
   if (p->num_splits > 1) {
     w.o_part = off;
     const size_t rows = static_cast<size_t>(p->total_q) * p->num_heads;
-    off = align256(off + rows * p->num_splits * p->head_size * sizeof(float));
+    off = align256(off + rows * p->num_splits * p->head_size * 2);  // fp16 partials
     w.lse_part = off;
     off = align256(off + rows * p->num_splits * sizeof(float));
   } else {
@@ -230,7 +230,7 @@ pa_status paged_attn_plan(const int32_t* cu_seqlens_q_host, const int32_t* seqle
   const double block_bytes = 2.0 * bs * cache_row_bytes(p->kv_dtype, p->head_size) *
                              (p->kv_num_heads < HP ? p->kv_num_heads : HP);
   const double item_cost = kItemCostBytes / block_bytes;
-  const double part_cost = 2.0 * HP * rows * p->head_size * 4.0 / block_bytes;
+  const double part_cost = 2.0 * HP * rows * (p->head_size * 2.0 + 4.0) / block_bytes;
   const int64_t slots = static_cast<int64_t>(sms) *
                         pa::forward_ctas_per_sm(p->kv_dtype, p->head_size, bs, rows);
   auto count = [&](int T, int64_t* items, int64_t* split_items, int* max_bps, int* max_ns,
@@ -347,7 +347,7 @@ pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_c
   a.err = reinterpret_cast<uint32_t*>(ws);
   a.work = reinterpret_cast<uint32_t*>(ws + pa::kWsWorkOffset);
   a.frag = reinterpret_cast<uint32_t*>(ws + lay.frag);
-  a.o_part = p->num_splits > 1 ? reinterpret_cast<float*>(ws + lay.o_part) : nullptr;
+  a.o_part = p->num_splits > 1 ? reinterpret_cast<__half*>(ws + lay.o_part) : nullptr;
   a.lse_part = p->num_splits > 1 ? reinterpret_cast<float*>(ws + lay.lse_part) : nullptr;
   a.batch = p->batch;
   a.H = p->num_heads;

@@ -1066,10 +1066,10 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
 #pragma unroll
           for (int mt = 0; mt < C::kMTiles; ++mt) {
             const int dd = out_dim<KV>(mt, g);
-            const float2 vs = __ldg(reinterpret_cast<const float2*>(vsc + dd));
-            const float o0 = o[nt][mt][j] * inv * vs.x;
-            const float o1 = o[nt][mt][j + 2] * inv * vs.y;
             if (!is_split) {
+              const float2 vs = __ldg(reinterpret_cast<const float2*>(vsc + dd));
+              const float o0 = o[nt][mt][j] * inv * vs.x;
+              const float o1 = o[nt][mt][j + 2] * inv * vs.y;
               if (a.out_bf16)
                 *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(a.out) +
                                                    orow * D + dd) = __floats2bfloat162_rn(o0, o1);
@@ -1077,7 +1077,10 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
                 *reinterpret_cast<__half2*>(reinterpret_cast<__half*>(a.out) + orow * D + dd) =
                     __floats2half2_rn(o0, o1);
             } else {
-              *reinterpret_cast<float2*>(a.o_part + prow * D + dd) = make_float2(o0, o1);
+              // the partial in code units (|o| <= max |code| <= 448): fp16 keeps
+              // it within 2^-12 of its range; the combine applies the V scale
+              *reinterpret_cast<__half2*>(a.o_part + prow * D + dd) =
+                  __floats2half2_rn(o[nt][mt][j] * inv, o[nt][mt][j + 2] * inv);
             }
           }
           if (is_split && g == 0)
@@ -1153,28 +1156,37 @@ __global__ void __launch_bounds__(128) pa_combine_kernel(const FwdArgs a) {
   // lane handles dims 4 lane .. 4 lane + 3
   constexpr int kD4 = D / 4;
   const bool dl = lane < kD4;
-  const float* base = a.o_part + static_cast<size_t>(gr) * D + 4 * (dl ? lane : 0);
+  const __half* base = a.o_part + static_cast<size_t>(gr) * D + 4 * (dl ? lane : 0);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int s8 = 0; s8 < S; s8 += 8) {
-    float4 v[8];
+    uint2 v[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u)
       v[u] = (s8 + u < S && dl)
-                 ? __ldcg(reinterpret_cast<const float4*>(base + (s8 + u) * stride * D))
-                 : make_float4(0.f, 0.f, 0.f, 0.f);
+                 ? __ldcg(reinterpret_cast<const uint2*>(base + (s8 + u) * stride * D))
+                 : make_uint2(0u, 0u);
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const int sp = s8 + u;
       const float wv = __shfl_sync(kFull, ls[(sp >> 5) & 3], sp & 31) * inv;
       if (sp < S) {
-        acc.x = fmaf(wv, v[u].x, acc.x);
-        acc.y = fmaf(wv, v[u].y, acc.y);
-        acc.z = fmaf(wv, v[u].z, acc.z);
-        acc.w = fmaf(wv, v[u].w, acc.w);
+        const float2 f01 = __half22float2(u2h2(v[u].x));
+        const float2 f23 = __half22float2(u2h2(v[u].y));
+        acc.x = fmaf(wv, f01.x, acc.x);
+        acc.y = fmaf(wv, f01.y, acc.y);
+        acc.z = fmaf(wv, f23.x, acc.z);
+        acc.w = fmaf(wv, f23.y, acc.w);
       }
     }
   }
   if (dl) {
+    // the V scale of the row's KV head
+    const float4 vs = __ldg(
+        reinterpret_cast<const float4*>(a.v_scale + static_cast<size_t>(hq / a.G) * D + 4 * lane));
+    acc.x *= vs.x;
+    acc.y *= vs.y;
+    acc.z *= vs.z;
+    acc.w *= vs.w;
     const size_t o = static_cast<size_t>(gr) * D + 4 * lane;
     if (a.out_bf16) {
       __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(a.out) + o);

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -18,7 +19,7 @@ struct FwdArgs {
   const int32_t* block_table;
   const int32_t* seqlens_k;
   const int32_t* cu_seqlens_q;
-  float* o_part;        // [max_splits, total_q * H, D] (split mode only)
+  __half* o_part;       // [max_splits, total_q * H, D] fp16, code units (split mode only)
   float* lse_part;      // [max_splits, total_q * H] (log2 domain)
   uint32_t* frag;       // [batch * Hk * num_row_groups] precomputed query fragment units
   uint32_t* work;       // [2]: next work item, CTAs finished (both rewound by the last CTA)
