@@ -48,7 +48,7 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Workspace layout shared by the planner and the forward call.
 struct WsLayout {
-  size_t frag, o_part, lse_part, total;
+  size_t frag, o_part, lse_part, row_ns, total;
 };
 
 WsLayout ws_layout(const paged_attn_params* p) {
@@ -64,8 +64,10 @@ WsLayout ws_layout(const paged_attn_params* p) {
     off = align256(off + rows * p->num_splits * p->head_size * 2);  // fp16 partials
     w.lse_part = off;
     off = align256(off + rows * p->num_splits * sizeof(float));
+    w.row_ns = off;  // each row's split count
+    off = align256(off + rows * sizeof(int32_t));
   } else {
-    w.o_part = w.lse_part = 0;
+    w.o_part = w.lse_part = w.row_ns = 0;
   }
   w.total = off;
   return w;
@@ -349,6 +351,7 @@ pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_c
   a.frag = reinterpret_cast<uint32_t*>(ws + lay.frag);
   a.o_part = p->num_splits > 1 ? reinterpret_cast<__half*>(ws + lay.o_part) : nullptr;
   a.lse_part = p->num_splits > 1 ? reinterpret_cast<float*>(ws + lay.lse_part) : nullptr;
+  a.row_ns = p->num_splits > 1 ? reinterpret_cast<int32_t*>(ws + lay.row_ns) : nullptr;
   a.batch = p->batch;
   a.H = p->num_heads;
   a.Hk = p->kv_num_heads;

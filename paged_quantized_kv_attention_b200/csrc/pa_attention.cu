@@ -229,46 +229,84 @@ __device__ __forceinline__ void query_fragments(const FwdArgs& a, const uint8_t*
                                                 float (&crow)[NT]) {
   using C = Cfg<KV, D, BS, NT, LP>;
   const int g = lane >> 2, tig = lane & 3;
+  // The thread's channels come in groups of kGS consecutive ones (INT4: 8, else
+  // 4), so its query and scale values arrive in a few vector loads, all issued
+  // before any arithmetic.  Group gi starts at channel
+  //   INT8: 32 (gi >> 1) + 16 (gi & 1) + 4 tig   INT4: 32 gi + 8 tig   FP8: 16 gi + 4 tig
+  // and its offset o is element 4 gi + o (INT8, FP8) or 8 gi + 4 (o & 1) + (o >> 1)
+  // (INT4) of the list above.  The four lanes of one g cover every channel.
+  constexpr int kN = D / 4;  // channels per lane
+  constexpr int kGS = (KV == PA_KV_INT4) ? 8 : 4;
+  constexpr int kNG = kN / kGS;
+  auto gbase = [&](int gi) {
+    if constexpr (KV == PA_KV_INT8) return 32 * (gi >> 1) + 16 * (gi & 1) + 4 * tig;
+    else if constexpr (KV == PA_KV_INT4) return 32 * gi + 8 * tig;
+    else return 16 * gi + 4 * tig;
+  };
+  auto elem = [](int gi, int o) {
+    return (KV == PA_KV_INT4) ? 8 * gi + 4 * (o & 1) + (o >> 1) : 4 * gi + o;
+  };
+  float sc[kN];  // k_scale of element i's channel
+#pragma unroll
+  for (int gi = 0; gi < kNG; ++gi)
+#pragma unroll
+    for (int k = 0; k < kGS / 4; ++k) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(sks + gbase(gi) + 4 * k));
+      sc[elem(gi, 4 * k + 0)] = v.x;
+      sc[elem(gi, 4 * k + 1)] = v.y;
+      sc[elem(gi, 4 * k + 2)] = v.z;
+      sc[elem(gi, 4 * k + 3)] = v.w;
+    }
+  uint32_t qraw[NT][kN / 2];  // 16-bit query values of group gi at words gi kGS / 2 ..
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int row = LP ? (g >> 1) : nt * 8 + g;
+    const int ru = row0 + row;
+    const bool valid = row < nrows;
+    const size_t roff = valid ? (static_cast<size_t>(ru / a.G) * a.H + ru % a.G) * D : 0;
+    const uint16_t* qr = reinterpret_cast<const uint16_t*>(qh) + roff;
+#pragma unroll
+    for (int gi = 0; gi < kNG; ++gi) {
+      if constexpr (kGS == 8) {
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (valid) v = __ldg(reinterpret_cast<const uint4*>(qr + gbase(gi)));
+        qraw[nt][4 * gi + 0] = v.x;
+        qraw[nt][4 * gi + 1] = v.y;
+        qraw[nt][4 * gi + 2] = v.z;
+        qraw[nt][4 * gi + 3] = v.w;
+      } else {
+        uint2 v = make_uint2(0u, 0u);
+        if (valid) v = __ldg(reinterpret_cast<const uint2*>(qr + gbase(gi)));
+        qraw[nt][2 * gi + 0] = v.x;
+        qraw[nt][2 * gi + 1] = v.y;
+      }
+    }
+  }
   float ksmax = 0.f;
 #pragma unroll
-  for (int d = lane; d < D; d += 32) ksmax = fmaxf(ksmax, fabsf(__ldg(sks + d)));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ksmax = fmaxf(ksmax, __shfl_xor_sync(kFull, ksmax, o));
+  for (int i = 0; i < kN; ++i) ksmax = fmaxf(ksmax, fabsf(sc[i]));
+  ksmax = fmaxf(ksmax, __shfl_xor_sync(kFull, ksmax, 1));
+  ksmax = fmaxf(ksmax, __shfl_xor_sync(kFull, ksmax, 2));
   if (!isfinite(ksmax) && lane == 0) record_error(a.err, PA_DEVERR_BAD_SCALE);
   int e_kv = 0;
   (void)frexpf(ksmax, &e_kv);
   const float f_kv = ldexpf(1.f, -e_kv);
+  const bool qbf = a.q_bf16;
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    const int row = LP ? (g >> 1) : nt * 8 + g;
-    const bool valid = row < nrows;
-    const int ru = row0 + row;
-    const size_t roff = valid ? (static_cast<size_t>(ru / a.G) * a.H + ru % a.G) * D : 0;
-    const __half* q16 = reinterpret_cast<const __half*>(qh) + roff;
-    const __nv_bfloat16* qbf = reinterpret_cast<const __nv_bfloat16*>(qh) + roff;
-    constexpr int kCh = 32;  // channels per lane (D = 128; 16 for D = 64)
-    constexpr int kN = D / 4;
     float w[kN];
     float rmax = 0.f;
 #pragma unroll
-    for (int i = 0; i < kN; ++i) {
-      int ch;
-      if constexpr (KV == PA_KV_INT8) {
-        const int s = i >> 3, r = (i >> 2) & 1, e = i & 3;
-        ch = 32 * s + 16 * r + 4 * tig + e;
-      } else if constexpr (KV == PA_KV_INT4) {
-        const int s = i >> 3, r = (i >> 2) & 1, e = i & 3;
-        ch = 32 * s + 8 * tig + 2 * e + r;
-      } else {
-        const int s = i >> 2, r = (i >> 1) & 1, e = i & 1;
-        ch = 16 * s + 4 * tig + 2 * r + e;
+    for (int gi = 0; gi < kNG; ++gi)
+#pragma unroll
+      for (int o = 0; o < kGS; ++o) {
+        const uint32_t bits = (qraw[nt][gi * kGS / 2 + o / 2] >> (16 * (o & 1))) & 0xFFFFu;
+        const float x = qbf ? __uint_as_float(bits << 16)
+                            : __half2float(__ushort_as_half(static_cast<unsigned short>(bits)));
+        const int i = elem(gi, o);
+        w[i] = x * (sc[i] * f_kv);
+        rmax = fmaxf(rmax, fabsf(w[i]));
       }
-      float x = 0.f;
-      if (valid) x = a.q_bf16 ? __bfloat162float(qbf[ch]) : __half2float(q16[ch]);
-      w[i] = x * (__ldg(sks + ch) * f_kv);
-      rmax = fmaxf(rmax, fabsf(w[i]));
-    }
-    (void)kCh;
     rmax = fmaxf(rmax, __shfl_xor_sync(kFull, rmax, 1));
     rmax = fmaxf(rmax, __shfl_xor_sync(kFull, rmax, 2));
     int e_q = 0;
@@ -333,15 +371,21 @@ __device__ __forceinline__ void query_fragments(const FwdArgs& a, const uint8_t*
 template <int KV, int D, int BS, int NT, bool LP>
 __global__ void __launch_bounds__(64) pa_prep_kernel(const FwdArgs a) {
   using C = Cfg<KV, D, BS, NT, LP>;
+  // This grid may be launched before the previous kernel of the stream has
+  // finished (programmatic launch): nothing is read or written before that
+  // grid's completion, and the forward kernel is released only after it.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;");
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2, tig = lane & 3;
-  const long long units = static_cast<long long>(a.batch) * a.Hk * a.num_row_groups;
-  const long long u = static_cast<long long>(blockIdx.x) * 2 + (threadIdx.x >> 5);
+  // unit (b, h, rg): the host keeps batch x Hk x row groups below 2^31
+  const int units = a.batch * a.Hk * a.num_row_groups;
+  const int u = blockIdx.x * 2 + (threadIdx.x >> 5);
   if (u >= units) return;
-  const int rg = static_cast<int>(u % a.num_row_groups);
-  const int h = static_cast<int>((u / a.num_row_groups) % a.Hk);
-  const int b = static_cast<int>(u / (static_cast<long long>(a.num_row_groups) * a.Hk));
+  const int bh = u / a.num_row_groups;
+  const int rg = u - bh * a.num_row_groups;
+  const int b = bh / a.Hk;
+  const int h = bh - b * a.Hk;
   const int q0 = __ldg(a.cu_seqlens_q + b), qb = __ldg(a.cu_seqlens_q + b + 1) - q0;
   const int Lb = __ldg(a.seqlens_k + b);
   if (qb <= 0 || qb > Lb || q0 < 0 || q0 + qb > a.total_q) return;
@@ -405,16 +449,34 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
   // may be scheduled onto SMs as this grid's CTAs finish; it waits for this
   // grid's completion before reading anything.
   asm volatile("griddepcontrol.launch_dependents;");
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
+  // The producer's first global reads, the sequence lengths (sequence 32 k + lane
+  // in register k, up to 256 sequences), go out before the barrier set-up.
+  constexpr int kMaxK = 8;
+  const int nk = (a.batch + 31) >> 5;
+  const bool dense = nk <= kMaxK;
+  int sq0[kMaxK], sq1[kMaxK], sL[kMaxK];
+  if (warp == C::kWarps && dense) {
+#pragma unroll
+    for (int k = 0; k < kMaxK; ++k) {
+      const int b = 32 * k + lane;
+      sq0[k] = sq1[k] = sL[k] = 0;
+      if (k < nk && b < a.batch) {
+        sq0[k] = __ldg(a.cu_seqlens_q + b);
+        sq1[k] = __ldg(a.cu_seqlens_q + b + 1);
+        sL[k] = __ldg(a.seqlens_k + b);
+      }
+    }
+  }
+  if (warp == 0) {  // one barrier per lane
+    for (int s = lane; s < C::kStages; s += 32) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), C::kWarps);
     }
-    for (int sl = 0; sl < 2; ++sl) {
-      mbar_init(item_full(sl), 1);
-      mbar_init(item_empty(sl), C::kWarps);
+    if (lane < 2) {
+      mbar_init(item_full(lane), 1);
+      mbar_init(item_empty(lane), C::kWarps);
     }
-    mbar_init(frag_ready, C::kWarps);
+    if (lane == 2) mbar_init(frag_ready, C::kWarps);
     mbar_fence_init();
   }
   __syncthreads();
@@ -426,43 +488,12 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
       tma_prefetch_desc(&vmap);
     }
     const uint64_t policy = l2_evict_first_policy();
-    // ---- L2 prefetch of what the first items read right after the lengths:
-    // the block table, the scale rows and the queries, each CTA a slice.
-    auto prefetch_slice = [&](const void* base, size_t bytes) {
-      const size_t lines = (bytes + 127) / 128;
-      const size_t per = (lines + gridDim.x - 1) / gridDim.x;
-      const size_t lo = blockIdx.x * per;
-      const size_t hi = lo + per < lines ? lo + per : lines;
-      for (size_t l = lo + lane; l < hi; l += 32) {
-        const size_t off = l * 128 < bytes ? l * 128 : bytes - 1;
-        prefetch_l2(reinterpret_cast<const uint8_t*>(base) + off);
-      }
-    };
-    prefetch_slice(a.block_table, static_cast<size_t>(a.batch) * a.maxb * 4);
-    prefetch_slice(a.k_scale, static_cast<size_t>(a.Hk) * D * 4);
-    prefetch_slice(a.v_scale, static_cast<size_t>(a.Hk) * D * 4);
-    prefetch_slice(a.q, static_cast<size_t>(a.total_q) * a.H * D * 2);
-    // ---- dense item numbering: per-sequence item counts and their prefix sums,
-    // sequence 32 k + lane in register k (up to 256 sequences); beyond that the
-    // numbering is sparse (every sequence gets the largest count; empty items
-    // are skipped).
-    constexpr int kMaxK = 8;
-    const int nk = (a.batch + 31) >> 5;
-    const bool dense = nk <= kMaxK;
-    int incl[kMaxK], cnt[kMaxK], sq0[kMaxK], sqb[kMaxK], sL[kMaxK];
+    // ---- dense item numbering: per-sequence item counts and their prefix sums
+    // (from the lengths loaded above); beyond 256 sequences the numbering is
+    // sparse (every sequence gets the largest count; empty items are skipped).
+    int incl[kMaxK], cnt[kMaxK];
     int total = 0, per_seq = 0;
     if (dense) {
-#pragma unroll
-      for (int k = 0; k < kMaxK; ++k) {
-        const int b = 32 * k + lane;
-        sq0[k] = sqb[k] = sL[k] = 0;
-        if (k < nk && b < a.batch) {
-          const int c0 = a.cu_seqlens_q[b], c1 = a.cu_seqlens_q[b + 1];
-          sq0[k] = c0;
-          sqb[k] = c1 - c0;
-          sL[k] = a.seqlens_k[b];
-        }
-      }
       bool bad_any = false;
 #pragma unroll
       for (int k = 0; k < kMaxK; ++k) {
@@ -470,8 +501,9 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
         cnt[k] = 0;
         if (k < nk) {  // warp-uniform
           bool bad = false;
+          sq1[k] -= sq0[k];  // new tokens
           cnt[k] = (32 * k + lane < a.batch)
-                       ? seq_items<BS>(a, rows_cta, sq0[k], sqb[k], sL[k], bad)
+                       ? seq_items<BS>(a, rows_cta, sq0[k], sq1[k], sL[k], bad)
                        : 0;
           bad_any |= bad;
           int x = cnt[k];
@@ -503,7 +535,7 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
             const int l = __ffs(m) - 1;
             const int base = __shfl_sync(kFull, incl[k] - cnt[k], l);
             const int q0 = __shfl_sync(kFull, sq0[k], l);
-            const int qb = __shfl_sync(kFull, sqb[k], l);
+            const int qb = __shfl_sync(kFull, sq1[k], l);
             const int Lb = __shfl_sync(kFull, sL[k], l);
             return decode_item<BS>(a, rows_cta, 32 * k + l, w - base, q0, qb, Lb, d);
           }
@@ -628,6 +660,18 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
           }
           ok = __shfl_sync(kFull, ok, l0);
         }
+      }
+      if (done == 0) {
+        // L2 prefetch of what later items and the epilogues read: the block
+        // table and the V scale rows, strided over the CTAs
+        auto prefetch_all = [&](const void* base, size_t bytes) {
+          const size_t step = static_cast<size_t>(gridDim.x) * 32 * 128;
+          for (size_t off = (static_cast<size_t>(blockIdx.x) * 32 + lane) * 128; off < bytes;
+               off += step)
+            prefetch_l2(reinterpret_cast<const uint8_t*>(base) + off);
+        };
+        prefetch_all(a.block_table, static_cast<size_t>(a.batch) * a.maxb * 4);
+        prefetch_all(a.v_scale, static_cast<size_t>(a.Hk) * D * 4);
       }
       done += nst;
       slot ^= 1;
@@ -1085,6 +1129,8 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
           }
           if (is_split && g == 0)
             a.lse_part[prow] = (L > 0.f) ? m_run[nt][j] + __log2f(L) : -INFINITY;
+          // every row's split count, for the combine (1: stored above)
+          if (a.row_ns != nullptr && split == 0 && g == 0) a.row_ns[orow] = nsplit;
         }
 
     }
@@ -1099,38 +1145,30 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
 // Log-sum-exp merge of the split partials (flash decoding, GQA GEMV decode page,
 // Code analysis 2: the workers' partials are combined after the split pass):
 //   lse = log2 sum_s 2^lse_s,  out = sum_s 2^(lse_s - lse) o_s
-// One warp per (new-token row, query head).  The warp recomputes, from the device
-// lengths and the plan, how many splits of its (sequence, KV head, row group)
-// have keys, exactly as the forward kernel decoded its items; rows of unsplit
-// units were stored by the forward kernel and are skipped.  Launched as the
-// forward kernel's programmatic dependent: it waits for the forward grid to
-// complete before reading a partial.
+// One warp per (new-token row, query head).  The forward kernel stored, for every
+// row, how many splits of its (sequence, KV head, row group) have keys; rows of
+// unsplit units (count 1) were stored by the forward kernel and are skipped.
+// Launched as the forward kernel's programmatic dependent: it waits for the
+// forward grid to complete before reading anything the forward grid wrote.
 template <int D, int BS>
 __global__ void __launch_bounds__(128) pa_combine_kernel(const FwdArgs a) {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int lane = threadIdx.x & 31;
   const int gr = blockIdx.x * 4 + (threadIdx.x >> 5);  // row of out viewed as [total_q * H]
-  if (gr >= a.total_q * a.H) return;
-  const int qrow = gr / a.H, hq = gr % a.H;
-  // sequence of the token: the last b with cu[b] <= qrow
-  int lo = 0, hi = a.batch - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(a.cu_seqlens_q + mid) <= qrow) lo = mid; else hi = mid - 1;
-  }
-  const int b = lo;
-  const int q0 = __ldg(a.cu_seqlens_q + b), qb = __ldg(a.cu_seqlens_q + b + 1) - q0;
-  const int Lb = __ldg(a.seqlens_k + b);
-  if (qb <= 0 || qb > Lb) return;
-  const int R = qb * a.G;
-  const int r = (qrow - q0) * a.G + hq % a.G;  // row within the (sequence, KV head) unit
-  const int row0 = (r / a.rows_cta) * a.rows_cta;
-  const int row_end = min(R, row0 + a.rows_cta);
-  const int i_last = (row_end - 1) / a.G;
-  const int kmax = a.causal ? (Lb - qb) + i_last + 1 : Lb;
-  int ns, bps;
-  split_geometry((Lb + BS - 1) / BS, a.split_target, a.max_splits, &ns, &bps);
-  const int S = ((kmax + BS - 1) / BS + bps - 1) / bps;
+  const bool row_ok = gr < a.total_q * a.H;
+  const int hq = row_ok ? gr % a.H : 0;
+  // the V scale of the row's KV head (an input: read before the wait)
+  constexpr int kD4 = D / 4;
+  const bool dl = lane < kD4;
+  float4 vs = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (row_ok && dl)
+    vs = __ldg(reinterpret_cast<const float4*>(a.v_scale + static_cast<size_t>(hq / a.G) * D +
+                                               4 * lane));
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // the next call's pre-pass may be scheduled now (it waits for this grid)
+  asm volatile("griddepcontrol.launch_dependents;");
+  if (!row_ok) return;
+  int S = __ldcg(a.row_ns + gr);
+  S = min(S, a.max_splits);  // a row of an invalid sequence holds no count of this call
   if (S <= 1) return;
   const size_t stride = static_cast<size_t>(a.total_q) * a.H;
   // weights 2^(lse_s - max) / sum; lane holds splits lane, lane + 32, ...
@@ -1154,8 +1192,6 @@ __global__ void __launch_bounds__(128) pa_combine_kernel(const FwdArgs a) {
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(kFull, sum, o);
   const float inv = sum > 0.f ? 1.f / sum : 0.f;
   // lane handles dims 4 lane .. 4 lane + 3
-  constexpr int kD4 = D / 4;
-  const bool dl = lane < kD4;
   const __half* base = a.o_part + static_cast<size_t>(gr) * D + 4 * (dl ? lane : 0);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int s8 = 0; s8 < S; s8 += 8) {
@@ -1180,9 +1216,6 @@ __global__ void __launch_bounds__(128) pa_combine_kernel(const FwdArgs a) {
     }
   }
   if (dl) {
-    // the V scale of the row's KV head
-    const float4 vs = __ldg(
-        reinterpret_cast<const float4*>(a.v_scale + static_cast<size_t>(hq / a.G) * D + 4 * lane));
     acc.x *= vs.x;
     acc.y *= vs.y;
     acc.z *= vs.z;
@@ -1261,10 +1294,23 @@ static cudaError_t launch_t(const CUtensorMap& kmap, const CUtensorMap& vmap, Fw
   const int grid = static_cast<int>(a.num_items < slots ? a.num_items : slots);
   if (grid < 1) return cudaSuccess;
   // the fragment pre-pass, then the forward kernel as its programmatic dependent
+  // the fragment pre-pass (a programmatic dependent of whatever precedes it in
+  // the stream: it waits for that grid before touching memory)
   const long long units = static_cast<long long>(a.batch) * a.Hk * a.num_row_groups;
-  pa_prep_kernel<KV, D, BS, NT, LP><<<static_cast<unsigned>((units + 1) / 2), 64, 0, stream>>>(a);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  if (units >= (1ll << 31)) return cudaErrorInvalidValue;
+  {
+    cudaLaunchConfig_t pc = {};
+    pc.gridDim = dim3(static_cast<unsigned>((units + 1) / 2));
+    pc.blockDim = dim3(64);
+    pc.stream = stream;
+    cudaLaunchAttribute pattr[1];
+    pattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pattr[0].val.programmaticStreamSerializationAllowed = 1;
+    pc.attrs = pattr;
+    pc.numAttrs = 1;
+    e = cudaLaunchKernelEx(&pc, pa_prep_kernel<KV, D, BS, NT, LP>, a);
+    if (e != cudaSuccess) return e;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(C::kThreads);

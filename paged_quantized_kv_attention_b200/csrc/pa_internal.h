@@ -21,6 +21,7 @@ struct FwdArgs {
   const int32_t* cu_seqlens_q;
   __half* o_part;       // [max_splits, total_q * H, D] fp16, code units (split mode only)
   float* lse_part;      // [max_splits, total_q * H] (log2 domain)
+  int32_t* row_ns;      // [total_q * H] splits with keys of each row's unit (split mode only)
   uint32_t* frag;       // [batch * Hk * num_row_groups] precomputed query fragment units
   uint32_t* work;       // [2]: next work item, CTAs finished (both rewound by the last CTA)
   uint32_t* err;        // sticky device error word
