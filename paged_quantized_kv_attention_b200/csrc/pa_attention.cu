@@ -527,20 +527,25 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
     auto locate = [&](int w, ItemDesc& d) -> bool {
       d.valid = 0;
       if (dense) {
+        // the first sequence whose inclusive prefix exceeds w (a small unrolled
+        // search with constant register indices, then one decode)
+        int fb = -1, fbase = 0, fq0 = 0, fqb = 0, fL = 0;
 #pragma unroll
         for (int k = 0; k < kMaxK; ++k) {
-          if (k >= nk) break;
-          const unsigned m = __ballot_sync(kFull, incl[k] > w);
-          if (m != 0u) {
-            const int l = __ffs(m) - 1;
-            const int base = __shfl_sync(kFull, incl[k] - cnt[k], l);
-            const int q0 = __shfl_sync(kFull, sq0[k], l);
-            const int qb = __shfl_sync(kFull, sq1[k], l);
-            const int Lb = __shfl_sync(kFull, sL[k], l);
-            return decode_item<BS>(a, rows_cta, 32 * k + l, w - base, q0, qb, Lb, d);
+          if (k < nk && fb < 0) {  // warp-uniform
+            const unsigned m = __ballot_sync(kFull, incl[k] > w);
+            if (m != 0u) {
+              const int l = __ffs(m) - 1;
+              fbase = __shfl_sync(kFull, incl[k] - cnt[k], l);
+              fq0 = __shfl_sync(kFull, sq0[k], l);
+              fqb = __shfl_sync(kFull, sq1[k], l);
+              fL = __shfl_sync(kFull, sL[k], l);
+              fb = 32 * k + l;
+            }
           }
         }
-        return false;
+        if (fb < 0) return false;
+        return decode_item<BS>(a, rows_cta, fb, w - fbase, fq0, fqb, fL, d);
       }
       const int b = w / per_seq;
       int v = 0;
@@ -568,7 +573,8 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
       return decode_item<BS>(a, rows_cta, b, (hg * rg_n + rg) * ns + split, q0, qb, Lb, d);
     };
 
-    int uses[2] = {0, 0};
+    int uses0 = 0, uses1 = 0;  // items published in slot 0 / 1
+    int fills = 0;             // copies issued into this lane's ring stage
     int slot = 0;
     int done = 0;  // stages issued so far: item stage kk lands in ring stage (done + kk) % kStages
     bool ok = true;
@@ -603,7 +609,8 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
       int phys = (owner && kk < nst) ? load_phys(kk) : 0;
       // publish the item (or the end marker) in the next slot
       if (lane == 0) {
-        if (uses[slot] > 0 && !mbar_wait(item_empty(slot), (uses[slot] - 1) & 1)) {
+        const int u = slot ? uses1 : uses0;
+        if (u > 0 && !mbar_wait(item_empty(slot), (u - 1) & 1)) {
           record_error(a.err, PA_DEVERR_TIMEOUT);
           ok = false;
         } else {
@@ -612,7 +619,7 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
         }
       }
       ok = __shfl_sync(kFull, ok, 0);
-      ++uses[slot];
+      if (slot) ++uses1; else ++uses0;
       if (!ok || !d.valid) break;
 
       // Each pass, every owner lane whose stage all four consumer warps have
@@ -636,6 +643,7 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
             mbar_arrive_expect_tx(full_bar(lane), C::kStageBytes);
             tma_load_3d(smem_u32(k_tile(lane)), &kmap, full_bar(lane), 0, tok, hrow, policy);
             tma_load_3d(smem_u32(v_tile(lane)), &vmap, full_bar(lane), 0, tok, hrow, policy);
+            ++fills;
             kk += C::kStages;
             if (kk < nst) phys = load_phys(kk);
             issued = true;
@@ -649,8 +657,13 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
           ok = __shfl_sync(kFull, ok, 0);
           gated = false;
         } else if (__ballot_sync(kFull, issued) == 0u) {
-          // nothing was free: sleep on the first pending lane's stage
-          const int l0 = __ffs(pend) - 1;
+          // Nothing was free: sleep on the oldest pending stage.  Its release
+          // needs no further issue (a consumer warp holds at most the two stages
+          // before it), whereas a younger stage's release can wait on the very
+          // stage this warp would then not be issuing.
+          const unsigned key = pending ? static_cast<unsigned>(kk) : 0xFFFFFFFFu;
+          const unsigned oldest = __reduce_min_sync(kFull, key);
+          const int l0 = __ffs(__ballot_sync(kFull, pending && key == oldest)) - 1;
           if (lane == l0) {
             const int round = (done + kk) / C::kStages;
             if (!mbar_wait(empty_bar(lane), (round - 1) & 1)) {
@@ -680,16 +693,15 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
     // The last prefetched index is consumed (its atomic has completed) before
     // this CTA signs off.
     const uint32_t last = __shfl_sync(kFull, w_pref, 0);
-    // Leave no copy in flight: wait for the last fill of every stage, all within
-    // one bounded window (the consumers normally consumed them already).
-    if (lane == 0) {
+    // Leave no copy in flight: every owner lane waits for the last fill it
+    // issued into its stage, all within one bounded window (the consumers
+    // normally consumed them already).
+    {
       const uint64_t deadline = global_timer_ns() + kWaitLimitNs;
-      bool fine = true;
-      for (int s = 0; fine && s < C::kStages && s < done; ++s) {
-        const int last_round = (done - 1 - s) / C::kStages;
-        fine = mbar_wait_until(full_bar((done - 1 - s) % C::kStages), last_round & 1, deadline);
-      }
-      if (!fine) record_error(a.err, PA_DEVERR_TIMEOUT);
+      const bool fine = fills == 0 || mbar_wait_until(full_bar(lane), (fills - 1) & 1, deadline);
+      if (__ballot_sync(kFull, !fine) != 0u && lane == 0) record_error(a.err, PA_DEVERR_TIMEOUT);
+    }
+    if (lane == 0) {
       if (last == 0xffffffffu) record_error(a.err, PA_DEVERR_BAD_LENGTH);  // (never: uses the value)
       __threadfence();
       // The last CTA to finish rewinds the work counter for the next call.
@@ -702,7 +714,7 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
   }
 
   // ======================================================== consumer warps
-  int uses[2] = {0, 0};
+  int uses0 = 0, uses1 = 0;  // items taken from slot 0 / 1
   int slot = 0;
   bool prep_done = false;  // the fragment pre-pass grid has completed
   int kc = 0;  // stages consumed so far: item stage it is ring stage (kc + it) % kStages
@@ -713,11 +725,11 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
   const int ld_chunk = lm >> 1;
 
   for (;;) {
-    if (!mbar_wait(item_full(slot), uses[slot] & 1)) {
+    if (!__all_sync(kFull, mbar_wait(item_full(slot), (slot ? uses1 : uses0) & 1))) {
       if (lane == 0) record_error(a.err, PA_DEVERR_TIMEOUT);
       break;
     }
-    ++uses[slot];
+    if (slot) ++uses1; else ++uses0;
     const ItemDesc d = descs[slot];
     if (!d.valid) break;
     const int h = d.hg * C::kHP + warp;  // this warp's KV head
@@ -727,7 +739,6 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
     const int blk_begin = d.blk_begin, nloc = d.nloc, nsplit = d.nsplit, Lb = d.Lb;
     const int nrows = row_end - row0;
     const int nst = nloc * C::kSPB;
-    bool alive = true;
 
     // ---- prologue: this head's precomputed query fragments and row multipliers
     // (written by the pre-pass kernel, which this grid waits for once)
@@ -801,131 +812,166 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
       }
     }
 
-    for (int it = 0; it < nst; ++it) {
-      const int s = (kc + it) % C::kStages, round = (kc + it) / C::kStages;
-      if (alive && !mbar_wait(full_bar(s), round & 1)) {
-        if (lane == 0) record_error(a.err, PA_DEVERR_TIMEOUT);
-        alive = false;
-      }
-      if (active && alive) {
-        const uint32_t kbase = smem_u32(k_tile(s) + warp * C::kHeadTile);
-        const uint32_t vbase = smem_u32(v_tile(s) + warp * C::kHeadTile);
-        const int key0 = (blk_begin + it / C::kSPB) * BS + (it % C::kSPB) * C::kTok;
-        const bool need_mask = key0 + 16 > kfull;
-
-        // ---------------- QK: X = logits (log2 units) minus the row's reference.
-        // LP: X[0][eh] = key g + 8 eh of row tig.  Else X[nt][e]: key g + 8 (e >> 1),
-        // row nt * 8 + 2 tig + (e & 1).
-        float X[NT][4];
-        if constexpr (C::kInt) {
-          int acc[C::kAcc][NT][4];
+    // Software-pipelined over stages: the QK products of stage it + 1 are issued
+    // before the softmax and PV of stage it, so the two dependency chains overlap.
+    // Xc holds the raw logits of stage it (LP: [0][0..1]).
+    float Xc[NT][4];
+    auto qk_stage = [&](int it, int s, float (&Xr)[NT][4]) {
+      const uint32_t kbase = smem_u32(k_tile(s) + warp * C::kHeadTile);
+      const int key0 = (blk_begin + it / C::kSPB) * BS + (it % C::kSPB) * C::kTok;
+      const bool need_mask = key0 + 16 > kfull;
 #pragma unroll
-          for (int i = 0; i < C::kAcc; ++i)
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) Xr[nt][e] = 0.f;
+      float (&X)[NT][4] = Xr;
+      // ---------------- QK: X = raw logits (log2 units).
+      // LP: X[0][eh] = key g + 8 eh of row tig.  Else X[nt][e]: key g + 8 (e >> 1),
+      // row nt * 8 + 2 tig + (e & 1).
+      if constexpr (C::kInt) {
+        int acc[C::kAcc][NT][4];
+#pragma unroll
+        for (int i = 0; i < C::kAcc; ++i)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[i][nt][e] = 0;
+#pragma unroll
+        for (int cp = 0; cp < C::kChunks / 2; ++cp) {
+          uint32_t r[4];
+          const uint32_t off = ld_row * C::kCHS + (2 * cp + ld_chunk) * 16;
+          ldsm_x4(kbase + swz<C::kSwzMask>(off), r);
+#pragma unroll
+          for (int hh = 0; hh < (KV == PA_KV_INT4 ? 2 : 1); ++hh) {
+            uint32_t a0, a1, a2, a3;
+            int ks;
+            if constexpr (KV == PA_KV_INT8) {
+              a0 = r[0]; a1 = r[1]; a2 = r[2]; a3 = r[3];  // 32 channels, raw codes
+              ks = cp;
+            } else {
+              // nibbles as signed bytes 16 x code: low nibbles shifted up, high masked
+              const uint32_t x0 = r[2 * hh], x1 = r[2 * hh + 1];  // keys g, g+8; chunk 2cp+hh
+              a0 = (x0 << 4) & 0xF0F0F0F0u;
+              a1 = (x1 << 4) & 0xF0F0F0F0u;
+              a2 = x0 & 0xF0F0F0F0u;
+              a3 = x1 & 0xF0F0F0F0u;
+              ks = 2 * cp + hh;
+            }
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-              for (int e = 0; e < 4; ++e) acc[i][nt][e] = 0;
-#pragma unroll
-          for (int cp = 0; cp < C::kChunks / 2; ++cp) {
-            uint32_t r[4];
-            const uint32_t off = ld_row * C::kCHS + (2 * cp + ld_chunk) * 16;
-            ldsm_x4(kbase + swz<C::kSwzMask>(off), r);
-#pragma unroll
-            for (int hh = 0; hh < (KV == PA_KV_INT4 ? 2 : 1); ++hh) {
-              uint32_t a0, a1, a2, a3;
-              int ks;
-              if constexpr (KV == PA_KV_INT8) {
-                a0 = r[0]; a1 = r[1]; a2 = r[2]; a3 = r[3];  // 32 channels, raw codes
-                ks = cp;
-              } else {
-                // nibbles as signed bytes 16 x code: low nibbles shifted up, high masked
-                const uint32_t x0 = r[2 * hh], x1 = r[2 * hh + 1];  // keys g, g+8; chunk 2cp+hh
-                a0 = (x0 << 4) & 0xF0F0F0F0u;
-                a1 = (x1 << 4) & 0xF0F0F0F0u;
-                a2 = x0 & 0xF0F0F0F0u;
-                a3 = x1 & 0xF0F0F0F0u;
-                ks = 2 * cp + hh;
-              }
-#pragma unroll
-              for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int i = 0; i < C::kAcc; ++i)
-                  imma_16832<false>(acc[i][nt], a0, a1, a2, a3, qf[nt][(ks * C::kAcc + i) * 2],
-                                    qf[nt][(ks * C::kAcc + i) * 2 + 1]);
-            }
-          }
-          if constexpr (LP) {
-#pragma unroll
-            for (int eh = 0; eh < 2; ++eh) {
-              const int A = acc[0][0][2 * eh] * 128 + acc[0][0][2 * eh + 1];
-              const int B2 = acc[1][0][2 * eh] * 128 + acc[1][0][2 * eh + 1];
-              float xv = fmaf(__int2float_rn(A), wA[0][0],
-                              fmaf(__int2float_rn(B2), wB[0][0], -msub[0][0]));
-              if (need_mask && key0 + g + 8 * eh > lim[0][0]) xv = -INFINITY;
-              X[0][eh] = xv;
-            }
-          } else {
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int j = e & 1;
-                const int A = acc[0][nt][e] * 128 + acc[1][nt][e];
-                float xv = fmaf(__int2float_rn(A), wA[nt][j],
-                                fmaf(__int2float_rn(acc[2][nt][e]), wB[nt][j], -msub[nt][j]));
-                if (need_mask && key0 + g + (e >> 1) * 8 > lim[nt][j]) xv = -INFINITY;
-                X[nt][e] = xv;
-              }
-          }
-        } else {
-          float sacc[C::kAcc][NT][4];
-#pragma unroll
-          for (int i = 0; i < C::kAcc; ++i)
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-              for (int e = 0; e < 4; ++e) sacc[i][nt][e] = 0.f;
-#pragma unroll
-          for (int cp = 0; cp < C::kChunks / 2; ++cp) {
-            uint32_t r[4];
-            const uint32_t off = ld_row * C::kCHS + (2 * cp + ld_chunk) * 16;
-            ldsm_x4(kbase + swz<C::kSwzMask>(off), r);
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              const int ks = 2 * cp + hh;  // 16-channel k-step
-              uint32_t a0, a1, a2, a3;
-              e4m3x4_to_h2x2(r[2 * hh], a0, a2);      // key g: channels +0,1 | +2,3
-              e4m3x4_to_h2x2(r[2 * hh + 1], a1, a3);  // key g+8
-#pragma unroll
-              for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int i = 0; i < C::kAcc; ++i)
-                  mma_16816(sacc[i][nt], a0, a1, a2, a3, qf[nt][(ks * C::kAcc + i) * 2],
-                            qf[nt][(ks * C::kAcc + i) * 2 + 1]);
-            }
-          }
-          if constexpr (LP) {
-#pragma unroll
-            for (int eh = 0; eh < 2; ++eh) {
-              // columns 2 tig / 2 tig + 1: high part / residual of row tig
-              float xv = fmaf(sacc[0][0][2 * eh] + sacc[0][0][2 * eh + 1], wA[0][0], -msub[0][0]);
-              if (need_mask && key0 + g + 8 * eh > lim[0][0]) xv = -INFINITY;
-              X[0][eh] = xv;
-            }
-          } else {
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int j = e & 1;
-                float xv = fmaf(sacc[0][nt][e] + sacc[1][nt][e], wA[nt][j], -msub[nt][j]);
-                if (need_mask && key0 + g + (e >> 1) * 8 > lim[nt][j]) xv = -INFINITY;
-                X[nt][e] = xv;
-              }
+              for (int i = 0; i < C::kAcc; ++i)
+                imma_16832<false>(acc[i][nt], a0, a1, a2, a3, qf[nt][(ks * C::kAcc + i) * 2],
+                                  qf[nt][(ks * C::kAcc + i) * 2 + 1]);
           }
         }
+        if constexpr (LP) {
+#pragma unroll
+          for (int eh = 0; eh < 2; ++eh) {
+            const int A = acc[0][0][2 * eh] * 128 + acc[0][0][2 * eh + 1];
+            const int B2 = acc[1][0][2 * eh] * 128 + acc[1][0][2 * eh + 1];
+            float xv = fmaf(__int2float_rn(A), wA[0][0], __int2float_rn(B2) * wB[0][0]);
+            if (need_mask && key0 + g + 8 * eh > lim[0][0]) xv = -INFINITY;
+            X[0][eh] = xv;
+          }
+        } else {
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int j = e & 1;
+              const int A = acc[0][nt][e] * 128 + acc[1][nt][e];
+              float xv = fmaf(__int2float_rn(A), wA[nt][j], __int2float_rn(acc[2][nt][e]) * wB[nt][j]);
+              if (need_mask && key0 + g + (e >> 1) * 8 > lim[nt][j]) xv = -INFINITY;
+              X[nt][e] = xv;
+            }
+        }
+      } else {
+        float sacc[C::kAcc][NT][4];
+#pragma unroll
+        for (int i = 0; i < C::kAcc; ++i)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sacc[i][nt][e] = 0.f;
+#pragma unroll
+        for (int cp = 0; cp < C::kChunks / 2; ++cp) {
+          uint32_t r[4];
+          const uint32_t off = ld_row * C::kCHS + (2 * cp + ld_chunk) * 16;
+          ldsm_x4(kbase + swz<C::kSwzMask>(off), r);
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int ks = 2 * cp + hh;  // 16-channel k-step
+            uint32_t a0, a1, a2, a3;
+            e4m3x4_to_h2x2(r[2 * hh], a0, a2);      // key g: channels +0,1 | +2,3
+            e4m3x4_to_h2x2(r[2 * hh + 1], a1, a3);  // key g+8
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+              for (int i = 0; i < C::kAcc; ++i)
+                mma_16816(sacc[i][nt], a0, a1, a2, a3, qf[nt][(ks * C::kAcc + i) * 2],
+                          qf[nt][(ks * C::kAcc + i) * 2 + 1]);
+          }
+        }
+        if constexpr (LP) {
+#pragma unroll
+          for (int eh = 0; eh < 2; ++eh) {
+            // columns 2 tig / 2 tig + 1: high part / residual of row tig
+            float xv = (sacc[0][0][2 * eh] + sacc[0][0][2 * eh + 1]) * wA[0][0];
+            if (need_mask && key0 + g + 8 * eh > lim[0][0]) xv = -INFINITY;
+            X[0][eh] = xv;
+          }
+        } else {
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int j = e & 1;
+              float xv = (sacc[0][nt][e] + sacc[1][nt][e]) * wA[nt][j];
+              if (need_mask && key0 + g + (e >> 1) * 8 > lim[nt][j]) xv = -INFINITY;
+              X[nt][e] = xv;
+            }
+        }
+      }
+    };
+    // Two n-tiles keep the stages sequential (registers).
+    constexpr bool kPipe = (NT == 1);
+    // A stage wait that gives up ends this warp (error flag set): it releases
+    // nothing more, so no stage is refilled while a copy into it may be in flight.
+    if (kPipe && nst > 0) {
+      if (!__all_sync(kFull, mbar_wait(full_bar(kc % C::kStages), (kc / C::kStages) & 1))) {
+        if (lane == 0) record_error(a.err, PA_DEVERR_TIMEOUT);
+        return;
+      }
+      if (active) qk_stage(0, kc % C::kStages, Xc);
+    }
+    for (int it = 0; it < nst; ++it) {
+      const int s = (kc + it) % C::kStages;
+      const bool has_next = it + 1 < nst;
+      const int sn = (kc + it + 1) % C::kStages;
+      const int sw = kPipe ? sn : s;  // the stage whose logits this pass computes
+      if ((kPipe ? has_next : true) &&
+          !__all_sync(kFull, mbar_wait(full_bar(sw), ((kc + it + (kPipe ? 1 : 0)) / C::kStages) & 1))) {
+        if (lane == 0) record_error(a.err, PA_DEVERR_TIMEOUT);
+        return;
+      }
+      if (active) {
+        // the next stage's logits (the last pass recomputes this stage's, unused),
+        // or, unpipelined, this stage's
+        float Xn[NT][4];
+        if constexpr (kPipe)
+          qk_stage(has_next ? it + 1 : it, has_next ? sn : s, Xn);
+        else
+          qk_stage(it, s, Xc);
+        const uint32_t vbase = smem_u32(v_tile(s) + warp * C::kHeadTile);
+        const int key0 = (blk_begin + it / C::kSPB) * BS + (it % C::kSPB) * C::kTok;
 
         // ---------------- online softmax with a lazily raised running max
+        float X[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) X[nt][e] = Xc[nt][e] - msub[nt][LP ? 0 : (e & 1)];
         if constexpr (LP) {
           float mx = fmaxf(X[0][0], X[0][1]);
           if (__any_sync(kFull, mx > thr[0][0])) {
@@ -1068,13 +1114,19 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
             }
           }
         }
+        if constexpr (kPipe) {
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) Xc[nt][e] = Xn[nt][e];
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(empty_bar(s));
     }
     kc += nst;
 
-    if (active && alive) {
+    if (active) {
       // ---- remove the code->fp16 constants (using the exact row sums of P);
       // accumulator columns j (LP: both = row tig)
 #pragma unroll
