@@ -54,6 +54,7 @@
 #include <math.h>
 
 #include <atomic>
+#include <type_traits>
 
 #include "pa_device.cuh"
 #include "pa_internal.h"
@@ -813,34 +814,26 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
     }
 
     // Software-pipelined over stages: the QK products of stage it + 1 are issued
-    // before the softmax and PV of stage it, so the two dependency chains overlap.
-    // Xc holds the raw logits of stage it (LP: [0][0..1]).
-    float Xc[NT][4];
-    auto qk_stage = [&](int it, int s, float (&Xr)[NT][4]) {
+    // before the softmax and PV of stage it and read only in the next pass, so
+    // their latency hides behind this stage's work.  Accumulator sets: integer
+    // digits (int) or FP8 parts (float).
+    using AccT = typename std::conditional<C::kInt, int, float>::type;
+    AccT accC[C::kAcc][NT][4], accN[C::kAcc][NT][4];
+    // QK products of ring stage s into acc (ldmatrix + MMA only).
+    auto qk_issue = [&](int s, AccT (&acc)[C::kAcc][NT][4]) {
       const uint32_t kbase = smem_u32(k_tile(s) + warp * C::kHeadTile);
-      const int key0 = (blk_begin + it / C::kSPB) * BS + (it % C::kSPB) * C::kTok;
-      const bool need_mask = key0 + 16 > kfull;
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
+      for (int i = 0; i < C::kAcc; ++i)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) Xr[nt][e] = 0.f;
-      float (&X)[NT][4] = Xr;
-      // ---------------- QK: X = raw logits (log2 units).
-      // LP: X[0][eh] = key g + 8 eh of row tig.  Else X[nt][e]: key g + 8 (e >> 1),
-      // row nt * 8 + 2 tig + (e & 1).
-      if constexpr (C::kInt) {
-        int acc[C::kAcc][NT][4];
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int i = 0; i < C::kAcc; ++i)
+          for (int e = 0; e < 4; ++e) acc[i][nt][e] = AccT(0);
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[i][nt][e] = 0;
-#pragma unroll
-        for (int cp = 0; cp < C::kChunks / 2; ++cp) {
-          uint32_t r[4];
-          const uint32_t off = ld_row * C::kCHS + (2 * cp + ld_chunk) * 16;
-          ldsm_x4(kbase + swz<C::kSwzMask>(off), r);
+      for (int cp = 0; cp < C::kChunks / 2; ++cp) {
+        uint32_t r[4];
+        const uint32_t off = ld_row * C::kCHS + (2 * cp + ld_chunk) * 16;
+        ldsm_x4(kbase + swz<C::kSwzMask>(off), r);
+        if constexpr (C::kInt) {
 #pragma unroll
           for (int hh = 0; hh < (KV == PA_KV_INT4 ? 2 : 1); ++hh) {
             uint32_t a0, a1, a2, a3;
@@ -864,41 +857,7 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
                 imma_16832<false>(acc[i][nt], a0, a1, a2, a3, qf[nt][(ks * C::kAcc + i) * 2],
                                   qf[nt][(ks * C::kAcc + i) * 2 + 1]);
           }
-        }
-        if constexpr (LP) {
-#pragma unroll
-          for (int eh = 0; eh < 2; ++eh) {
-            const int A = acc[0][0][2 * eh] * 128 + acc[0][0][2 * eh + 1];
-            const int B2 = acc[1][0][2 * eh] * 128 + acc[1][0][2 * eh + 1];
-            float xv = fmaf(__int2float_rn(A), wA[0][0], __int2float_rn(B2) * wB[0][0]);
-            if (need_mask && key0 + g + 8 * eh > lim[0][0]) xv = -INFINITY;
-            X[0][eh] = xv;
-          }
         } else {
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int j = e & 1;
-              const int A = acc[0][nt][e] * 128 + acc[1][nt][e];
-              float xv = fmaf(__int2float_rn(A), wA[nt][j], __int2float_rn(acc[2][nt][e]) * wB[nt][j]);
-              if (need_mask && key0 + g + (e >> 1) * 8 > lim[nt][j]) xv = -INFINITY;
-              X[nt][e] = xv;
-            }
-        }
-      } else {
-        float sacc[C::kAcc][NT][4];
-#pragma unroll
-        for (int i = 0; i < C::kAcc; ++i)
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) sacc[i][nt][e] = 0.f;
-#pragma unroll
-        for (int cp = 0; cp < C::kChunks / 2; ++cp) {
-          uint32_t r[4];
-          const uint32_t off = ld_row * C::kCHS + (2 * cp + ld_chunk) * 16;
-          ldsm_x4(kbase + swz<C::kSwzMask>(off), r);
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
             const int ks = 2 * cp + hh;  // 16-channel k-step
@@ -909,33 +868,58 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
               for (int i = 0; i < C::kAcc; ++i)
-                mma_16816(sacc[i][nt], a0, a1, a2, a3, qf[nt][(ks * C::kAcc + i) * 2],
+                mma_16816(acc[i][nt], a0, a1, a2, a3, qf[nt][(ks * C::kAcc + i) * 2],
                           qf[nt][(ks * C::kAcc + i) * 2 + 1]);
           }
         }
-        if constexpr (LP) {
-#pragma unroll
-          for (int eh = 0; eh < 2; ++eh) {
-            // columns 2 tig / 2 tig + 1: high part / residual of row tig
-            float xv = (sacc[0][0][2 * eh] + sacc[0][0][2 * eh + 1]) * wA[0][0];
-            if (need_mask && key0 + g + 8 * eh > lim[0][0]) xv = -INFINITY;
-            X[0][eh] = xv;
-          }
-        } else {
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int j = e & 1;
-              float xv = (sacc[0][nt][e] + sacc[1][nt][e]) * wA[nt][j];
-              if (need_mask && key0 + g + (e >> 1) * 8 > lim[nt][j]) xv = -INFINITY;
-              X[nt][e] = xv;
-            }
-        }
       }
     };
-    // Two n-tiles keep the stages sequential (registers).
-    constexpr bool kPipe = (NT == 1);
+    // Raw logits (log2 units) of item stage it from its products, masked.
+    // LP: X[0][eh] = key g + 8 eh of row tig.  Else X[nt][e]: key g + 8 (e >> 1),
+    // row nt * 8 + 2 tig + (e & 1).
+    auto qk_finish = [&](int it, const AccT (&acc)[C::kAcc][NT][4], float (&X)[NT][4]) {
+      const int key0 = (blk_begin + it / C::kSPB) * BS + (it % C::kSPB) * C::kTok;
+      const bool need_mask = key0 + 16 > kfull;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) X[nt][e] = 0.f;
+      if constexpr (LP) {
+#pragma unroll
+        for (int eh = 0; eh < 2; ++eh) {
+          float xv;
+          if constexpr (C::kInt) {
+            const int A = acc[0][0][2 * eh] * 128 + acc[0][0][2 * eh + 1];
+            const int B2 = acc[1][0][2 * eh] * 128 + acc[1][0][2 * eh + 1];
+            xv = fmaf(__int2float_rn(A), wA[0][0], __int2float_rn(B2) * wB[0][0]);
+          } else {
+            // columns 2 tig / 2 tig + 1: high part / residual of row tig
+            xv = (float(acc[0][0][2 * eh]) + float(acc[0][0][2 * eh + 1])) * wA[0][0];
+          }
+          if (need_mask && key0 + g + 8 * eh > lim[0][0]) xv = -INFINITY;
+          X[0][eh] = xv;
+        }
+      } else {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = e & 1;
+            float xv;
+            if constexpr (C::kInt) {
+              const int A = acc[0][nt][e] * 128 + acc[1][nt][e];
+              xv = fmaf(__int2float_rn(A), wA[nt][j], __int2float_rn(acc[2 % C::kAcc][nt][e]) * wB[nt][j]);
+            } else {
+              xv = (float(acc[0][nt][e]) + float(acc[1 % C::kAcc][nt][e])) * wA[nt][j];
+            }
+            if (need_mask && key0 + g + (e >> 1) * 8 > lim[nt][j]) xv = -INFINITY;
+            X[nt][e] = xv;
+          }
+      }
+    };
+    // Two n-tiles, and FP8 with two parts per row, keep the stages sequential
+    // (registers).
+    constexpr bool kPipe = (NT == 1) && (C::kInt || LP);
     // A stage wait that gives up ends this warp (error flag set): it releases
     // nothing more, so no stage is refilled while a copy into it may be in flight.
     if (kPipe && nst > 0) {
@@ -943,7 +927,7 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
         if (lane == 0) record_error(a.err, PA_DEVERR_TIMEOUT);
         return;
       }
-      if (active) qk_stage(0, kc % C::kStages, Xc);
+      if (active) qk_issue(kc % C::kStages, accN);
     }
     for (int it = 0; it < nst; ++it) {
       const int s = (kc + it) % C::kStages;
@@ -956,13 +940,22 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
         return;
       }
       if (active) {
-        // the next stage's logits (the last pass recomputes this stage's, unused),
-        // or, unpipelined, this stage's
-        float Xn[NT][4];
-        if constexpr (kPipe)
-          qk_stage(has_next ? it + 1 : it, has_next ? sn : s, Xn);
-        else
-          qk_stage(it, s, Xc);
+        // this stage's logits from the products issued last pass, then the next
+        // stage's products (the last pass reissues this stage's, unused); or,
+        // unpipelined, this stage's products and logits
+        float Xc[NT][4];
+        if constexpr (kPipe) {
+#pragma unroll
+          for (int i = 0; i < C::kAcc; ++i)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) accC[i][nt][e] = accN[i][nt][e];
+          qk_issue(has_next ? sn : s, accN);
+        } else {
+          qk_issue(s, accC);
+        }
+        qk_finish(it, accC, Xc);
         const uint32_t vbase = smem_u32(v_tile(s) + warp * C::kHeadTile);
         const int key0 = (blk_begin + it / C::kSPB) * BS + (it % C::kSPB) * C::kTok;
 
@@ -1114,12 +1107,6 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
             }
           }
         }
-        if constexpr (kPipe) {
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) Xc[nt][e] = Xn[nt][e];
-        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(empty_bar(s));
@@ -1197,39 +1184,60 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
 // Log-sum-exp merge of the split partials (flash decoding, GQA GEMV decode page,
 // Code analysis 2: the workers' partials are combined after the split pass):
 //   lse = log2 sum_s 2^lse_s,  out = sum_s 2^(lse_s - lse) o_s
-// One warp per (new-token row, query head).  The forward kernel stored, for every
-// row, how many splits of its (sequence, KV head, row group) have keys; rows of
-// unsplit units (count 1) were stored by the forward kernel and are skipped.
-// Launched as the forward kernel's programmatic dependent: it waits for the
-// forward grid to complete before reading anything the forward grid wrote.
-template <int D, int BS>
+// WPR warps per (new-token row, query head): four when the rows are few (one
+// CTA per row; warp w takes splits w, w + 4, ...), else one (four rows per CTA).
+// The forward kernel stored, for every row, how many splits of its (sequence,
+// KV head, row group) have keys; rows of unsplit units (count 1) were stored by
+// the forward kernel and are skipped.  Every load the merge needs goes out in
+// one round trip after the wait: the count, the log-sum-exps of all planned
+// splits and the partials of the warp's first splits; values of splits past
+// the row's count are never used.  Launched as the forward kernel's
+// programmatic dependent: it waits for the forward grid to complete before
+// reading anything the forward grid wrote.
+template <int D, int BS, int WPR>
 __global__ void __launch_bounds__(128) pa_combine_kernel(const FwdArgs a) {
-  const int lane = threadIdx.x & 31;
-  const int gr = blockIdx.x * 4 + (threadIdx.x >> 5);  // row of out viewed as [total_q * H]
+  __shared__ float4 red[3][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int wsub = warp % WPR;                        // this warp's share of the splits
+  const int gr = blockIdx.x * (4 / WPR) + warp / WPR;  // row of out viewed as [total_q * H]
   const bool row_ok = gr < a.total_q * a.H;
   const int hq = row_ok ? gr % a.H : 0;
-  // the V scale of the row's KV head (an input: read before the wait)
-  constexpr int kD4 = D / 4;
+  constexpr int kD4 = D / 4;  // lane handles dims 4 lane .. 4 lane + 3
   const bool dl = lane < kD4;
+  const int P = a.max_splits;  // planned splits (partials allocated per split)
+  // the V scale of the row's KV head (an input: read before the wait)
   float4 vs = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (row_ok && dl)
+  if (row_ok && wsub == 0 && dl)
     vs = __ldg(reinterpret_cast<const float4*>(a.v_scale + static_cast<size_t>(hq / a.G) * D +
                                                4 * lane));
   asm volatile("griddepcontrol.wait;" ::: "memory");
   // the next call's pre-pass may be scheduled now (it waits for this grid)
   asm volatile("griddepcontrol.launch_dependents;");
-  if (!row_ok) return;
-  int S = __ldcg(a.row_ns + gr);
-  S = min(S, a.max_splits);  // a row of an invalid sequence holds no count of this call
-  if (S <= 1) return;
+  if (!row_ok) return;  // warp-uniform; a whole CTA when WPR = 4
   const size_t stride = static_cast<size_t>(a.total_q) * a.H;
-  // weights 2^(lse_s - max) / sum; lane holds splits lane, lane + 32, ...
+  int S = __ldcg(a.row_ns + gr);
   float ls[4];
-  float M = -INFINITY;
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int sp = lane + 32 * k;
-    ls[k] = sp < S ? __ldcg(a.lse_part + sp * stride + gr) : -INFINITY;
+    ls[k] = sp < P ? __ldcg(a.lse_part + sp * stride + gr) : -INFINITY;
+  }
+  constexpr int kB = 8;  // partials in flight per lane
+  const __half* base = a.o_part + static_cast<size_t>(gr) * D + 4 * (dl ? lane : 0);
+  uint2 v[kB];
+#pragma unroll
+  for (int u = 0; u < kB; ++u) {
+    const int sp = wsub + WPR * u;
+    v[u] = (sp < P && dl) ? __ldcg(reinterpret_cast<const uint2*>(base + sp * stride * D))
+                          : make_uint2(0u, 0u);
+  }
+  S = min(S, P);  // a row of an invalid sequence holds no count of this call
+  if (S <= 1) return;  // uniform over the row's warps
+  // weights 2^(lse_s - max) / sum over the row's splits
+  float M = -INFINITY;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    if (lane + 32 * k >= S) ls[k] = -INFINITY;
     M = fmaxf(M, ls[k]);
   }
 #pragma unroll
@@ -1243,19 +1251,19 @@ __global__ void __launch_bounds__(128) pa_combine_kernel(const FwdArgs a) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(kFull, sum, o);
   const float inv = sum > 0.f ? 1.f / sum : 0.f;
-  // lane handles dims 4 lane .. 4 lane + 3
-  const __half* base = a.o_part + static_cast<size_t>(gr) * D + 4 * (dl ? lane : 0);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s8 = 0; s8 < S; s8 += 8) {
-    uint2 v[8];
+  for (int u0 = 0; wsub + WPR * u0 < S; u0 += kB) {
+    if (u0 > 0) {  // splits beyond the first batch
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
-      v[u] = (s8 + u < S && dl)
-                 ? __ldcg(reinterpret_cast<const uint2*>(base + (s8 + u) * stride * D))
-                 : make_uint2(0u, 0u);
+      for (int u = 0; u < kB; ++u) {
+        const int sp = wsub + WPR * (u0 + u);
+        v[u] = (sp < S && dl) ? __ldcg(reinterpret_cast<const uint2*>(base + sp * stride * D))
+                              : make_uint2(0u, 0u);
+      }
+    }
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int sp = s8 + u;
+    for (int u = 0; u < kB; ++u) {
+      const int sp = wsub + WPR * (u0 + u);
       const float wv = __shfl_sync(kFull, ls[(sp >> 5) & 3], sp & 31) * inv;
       if (sp < S) {
         const float2 f01 = __half22float2(u2h2(v[u].x));
@@ -1267,30 +1275,46 @@ __global__ void __launch_bounds__(128) pa_combine_kernel(const FwdArgs a) {
       }
     }
   }
-  if (dl) {
-    acc.x *= vs.x;
-    acc.y *= vs.y;
-    acc.z *= vs.z;
-    acc.w *= vs.w;
-    const size_t o = static_cast<size_t>(gr) * D + 4 * lane;
-    if (a.out_bf16) {
-      __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(a.out) + o);
-      dst[0] = __floats2bfloat162_rn(acc.x, acc.y);
-      dst[1] = __floats2bfloat162_rn(acc.z, acc.w);
-    } else {
-      __half2* dst = reinterpret_cast<__half2*>(reinterpret_cast<__half*>(a.out) + o);
-      dst[0] = __floats2half2_rn(acc.x, acc.y);
-      dst[1] = __floats2half2_rn(acc.z, acc.w);
+  if constexpr (WPR > 1) {  // the four warps' sums
+    if (warp > 0) red[warp - 1][lane] = acc;
+    __syncthreads();
+    if (warp != 0) return;
+#pragma unroll
+    for (int w = 0; w < 3; ++w) {
+      const float4 t = red[w][lane];
+      acc.x += t.x;
+      acc.y += t.y;
+      acc.z += t.z;
+      acc.w += t.w;
     }
   }
+  if (!dl) return;
+  acc.x *= vs.x;
+  acc.y *= vs.y;
+  acc.z *= vs.z;
+  acc.w *= vs.w;
+  const size_t o = static_cast<size_t>(gr) * D + 4 * lane;
+  if (a.out_bf16) {
+    __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(a.out) + o);
+    dst[0] = __floats2bfloat162_rn(acc.x, acc.y);
+    dst[1] = __floats2bfloat162_rn(acc.z, acc.w);
+  } else {
+    __half2* dst = reinterpret_cast<__half2*>(reinterpret_cast<__half*>(a.out) + o);
+    dst[0] = __floats2half2_rn(acc.x, acc.y);
+    dst[1] = __floats2half2_rn(acc.z, acc.w);
+  }
 }
+
+// Rows below this count get four warps each (one CTA per row).
+constexpr long long kCombineSplitWarpRows = 1024;
 
 template <int D, int BS>
 static cudaError_t launch_combine_t(const FwdArgs& a, cudaStream_t stream) {
   const long long rows = static_cast<long long>(a.total_q) * a.H;
   if (rows <= 0) return cudaSuccess;
+  const bool few = rows < kCombineSplitWarpRows;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>((rows + 3) / 4));
+  cfg.gridDim = dim3(static_cast<unsigned>(few ? rows : (rows + 3) / 4));
   cfg.blockDim = dim3(128);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
@@ -1299,7 +1323,8 @@ static cudaError_t launch_combine_t(const FwdArgs& a, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, pa_combine_kernel<D, BS>, a);
+  return few ? cudaLaunchKernelEx(&cfg, pa_combine_kernel<D, BS, 4>, a)
+             : cudaLaunchKernelEx(&cfg, pa_combine_kernel<D, BS, 1>, a);
 }
 
 cudaError_t launch_combine(int head_size, int block_size, const FwdArgs& a, cudaStream_t stream) {
@@ -1334,7 +1359,12 @@ static cudaError_t launch_t(const CUtensorMap& kmap, const CUtensorMap& vmap, Fw
                              cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(pa_combine_kernel<D, BS>, cudaFuncAttributePreferredSharedMemoryCarveout,
+    e = cudaFuncSetAttribute(pa_combine_kernel<D, BS, 1>,
+                             cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(pa_combine_kernel<D, BS, 4>,
+                             cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, C::kThreads, C::kSmemBytes);
