@@ -104,12 +104,18 @@ struct Cfg {
   static constexpr int kBarOff = kRingBytes;
   static constexpr int kNumBars = 2 * kStages + 5;  // full, empty, item full/empty x2, fragments
   static constexpr int kDescOff = kBarOff + kNumBars * 8;
-  static constexpr int kSmemBytes = kDescOff + 2 * 64;
+  // the producer's item table: inclusive item prefix per sequence, for as many
+  // sequences (a multiple of 32, at most 256) as the budget leaves room for
+  static constexpr int kTableOff = kDescOff + 2 * 64;
+  static constexpr int kTableRoom = (kBudget + 1024 - kTableOff) / 4;
+  static constexpr int kTableSeqs = (kTableRoom >= 256 ? 256 : kTableRoom) / 32 * 32;
+  static constexpr int kSmemBytes = kTableOff + kTableSeqs * 4;
   static_assert(kChunks % 2 == 0, "ldmatrix.x4 covers two 16-byte chunks");
   static_assert(kHeadTile % ((kSwzMask + 1) * 128) == 0, "tiles keep the swizzle-atom alignment");
   static_assert(kStages <= 32, "one producer lane per stage");
   static_assert(BS % kTok == 0, "whole stages per block");
   static_assert(kSmemBytes <= kBudget + 1024, "shared memory budget");
+  static_assert(kTableSeqs >= 32, "item table holds at least one warp of sequences");
 };
 
 // One work item as published by the producer to the consumers (64 bytes).
@@ -450,23 +456,15 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
   // may be scheduled onto SMs as this grid's CTAs finish; it waits for this
   // grid's completion before reading anything.
   asm volatile("griddepcontrol.launch_dependents;");
-  // The producer's first global reads, the sequence lengths (sequence 32 k + lane
-  // in register k, up to 256 sequences), go out before the barrier set-up.
-  constexpr int kMaxK = 8;
+  // The producer's first global reads, the lengths of sequences 0..31 (lane b),
+  // go out before the barrier set-up.
   const int nk = (a.batch + 31) >> 5;
-  const bool dense = nk <= kMaxK;
-  int sq0[kMaxK], sq1[kMaxK], sL[kMaxK];
-  if (warp == C::kWarps && dense) {
-#pragma unroll
-    for (int k = 0; k < kMaxK; ++k) {
-      const int b = 32 * k + lane;
-      sq0[k] = sq1[k] = sL[k] = 0;
-      if (k < nk && b < a.batch) {
-        sq0[k] = __ldg(a.cu_seqlens_q + b);
-        sq1[k] = __ldg(a.cu_seqlens_q + b + 1);
-        sL[k] = __ldg(a.seqlens_k + b);
-      }
-    }
+  const bool dense = a.batch <= C::kTableSeqs;
+  int f_q0 = 0, f_q1 = 0, f_L = 0;
+  if (warp == C::kWarps && dense && lane < a.batch) {
+    f_q0 = __ldg(a.cu_seqlens_q + lane);
+    f_q1 = __ldg(a.cu_seqlens_q + lane + 1);
+    f_L = __ldg(a.seqlens_k + lane);
   }
   if (warp == 0) {  // one barrier per lane
     for (int s = lane; s < C::kStages; s += 32) {
@@ -490,33 +488,37 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
     }
     const uint64_t policy = l2_evict_first_policy();
     // ---- dense item numbering: per-sequence item counts and their prefix sums
-    // (from the lengths loaded above); beyond 256 sequences the numbering is
-    // sparse (every sequence gets the largest count; empty items are skipped).
-    int incl[kMaxK], cnt[kMaxK];
+    // in shared memory (compact rolled loops: this runs once per CTA on a cold
+    // instruction cache); beyond kTableSeqs sequences the numbering is sparse
+    // (every sequence gets the largest count; empty items are skipped).
+    int* s_incl = reinterpret_cast<int*>(smem + C::kTableOff);
     int total = 0, per_seq = 0;
     if (dense) {
       bool bad_any = false;
-#pragma unroll
-      for (int k = 0; k < kMaxK; ++k) {
-        incl[k] = total;
-        cnt[k] = 0;
-        if (k < nk) {  // warp-uniform
-          bool bad = false;
-          sq1[k] -= sq0[k];  // new tokens
-          cnt[k] = (32 * k + lane < a.batch)
-                       ? seq_items<BS>(a, rows_cta, sq0[k], sq1[k], sL[k], bad)
-                       : 0;
-          bad_any |= bad;
-          int x = cnt[k];
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(kFull, x, o);
-            if (lane >= o) x += y;
+#pragma unroll 1
+      for (int k = 0; k < nk; ++k) {
+        const int b = 32 * k + lane;
+        int q0 = f_q0, q1 = f_q1, L = f_L;
+        if (k > 0) {
+          q0 = q1 = L = 0;
+          if (b < a.batch) {
+            q0 = __ldg(a.cu_seqlens_q + b);
+            q1 = __ldg(a.cu_seqlens_q + b + 1);
+            L = __ldg(a.seqlens_k + b);
           }
-          incl[k] = total + x;
-          total += __shfl_sync(kFull, x, 31);
         }
+        bool bad = false;
+        int x = b < a.batch ? seq_items<BS>(a, rows_cta, q0, q1 - q0, L, bad) : 0;
+        bad_any |= bad;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(kFull, x, o);
+          if (lane >= o) x += y;
+        }
+        s_incl[b] = total + x;  // b < 32 nk <= kTableSeqs
+        total += __shfl_sync(kFull, x, 31);
       }
+      __syncwarp();
       if (bad_any) record_error(a.err, PA_DEVERR_BAD_LENGTH);
     } else {
       per_seq = head_groups(a) * a.num_row_groups * a.max_splits;
@@ -528,25 +530,20 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
     auto locate = [&](int w, ItemDesc& d) -> bool {
       d.valid = 0;
       if (dense) {
-        // the first sequence whose inclusive prefix exceeds w (a small unrolled
-        // search with constant register indices, then one decode)
-        int fb = -1, fbase = 0, fq0 = 0, fqb = 0, fL = 0;
-#pragma unroll
-        for (int k = 0; k < kMaxK; ++k) {
-          if (k < nk && fb < 0) {  // warp-uniform
-            const unsigned m = __ballot_sync(kFull, incl[k] > w);
-            if (m != 0u) {
-              const int l = __ffs(m) - 1;
-              fbase = __shfl_sync(kFull, incl[k] - cnt[k], l);
-              fq0 = __shfl_sync(kFull, sq0[k], l);
-              fqb = __shfl_sync(kFull, sq1[k], l);
-              fL = __shfl_sync(kFull, sL[k], l);
-              fb = 32 * k + l;
-            }
-          }
+        // the first sequence whose inclusive prefix exceeds w
+        int fb = -1;
+#pragma unroll 1
+        for (int k = 0; k < nk && fb < 0; ++k) {
+          const int b = 32 * k + lane;
+          const unsigned m = __ballot_sync(kFull, b < a.batch && s_incl[b] > w);
+          if (m != 0u) fb = 32 * k + __ffs(m) - 1;
         }
         if (fb < 0) return false;
-        return decode_item<BS>(a, rows_cta, fb, w - fbase, fq0, fqb, fL, d);
+        const int base = fb > 0 ? s_incl[fb - 1] : 0;
+        const int q0 = __ldg(a.cu_seqlens_q + fb);
+        const int qb = __ldg(a.cu_seqlens_q + fb + 1) - q0;
+        const int Lb = __ldg(a.seqlens_k + fb);
+        return decode_item<BS>(a, rows_cta, fb, w - base, q0, qb, Lb, d);
       }
       const int b = w / per_seq;
       int v = 0;
