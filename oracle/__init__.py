@@ -56,6 +56,8 @@ def _load():
         _lib.oracle_decode.restype = ctypes.c_double
         _lib.oracle_pack_int4.argtypes = [P, ctypes.c_int64, ctypes.c_int, P]
         _lib.oracle_unpack_int4.argtypes = [P, ctypes.c_int64, ctypes.c_int, P]
+        _lib.oracle_quantise.argtypes = [ctypes.c_int, ctypes.c_float, ctypes.c_float]
+        _lib.oracle_append.argtypes = [ctypes.POINTER(_Problem)] + [P] * 9
         for fn in (_lib.oracle_paged_attn, _lib.oracle_paged_attn_folded):
             fn.argtypes = [ctypes.POINTER(_Problem)] + [P] * 9
         _lib.oracle_paged_attn_partial.argtypes = [ctypes.POINTER(_Problem)] + [P] * 12
@@ -175,3 +177,25 @@ def gather_decode(w: dict, cache: np.ndarray, b: int, kv: int) -> np.ndarray:
     if rc != 0:
         raise ValueError("oracle rejected the gather")
     return out
+
+
+def quantise(kv_dtype: int, x: float, s: float) -> int:
+    """Cache code of value x under scale s (signed code for INT8/INT4, byte for FP8)."""
+    return int(_load().oracle_quantise(kv_dtype, float(x), float(s)))
+
+
+def append(w: dict, k_new: np.ndarray, v_new: np.ndarray):
+    """Quantise-and-append: copies of w's k_cache / v_cache with the new rows
+    k_new / v_new ([T_q, Hk, D], exact values) written at their slots."""
+    lib = _load()
+    kc = np.array(w["k_cache"], dtype=np.uint8, copy=True, order="C")
+    vc = np.array(w["v_cache"], dtype=np.uint8, copy=True, order="C")
+    kn, vn = _c(k_new, np.float64), _c(v_new, np.float64)
+    ks, vs = _c(w["k_scale"], np.float32), _c(w["v_scale"], np.float32)
+    bt, sk, cq = _c(w["block_table"], np.int32), _c(w["seqlens_k"], np.int32), _c(
+        w["cu_seqlens_q"], np.int32)
+    rc = lib.oracle_append(ctypes.byref(_problem(w)), _ptr(kn), _ptr(vn), _ptr(ks), _ptr(vs),
+                           _ptr(bt), _ptr(sk), _ptr(cq), _ptr(kc), _ptr(vc))
+    if rc != 0:
+        raise ValueError("oracle rejected the problem (contract violation)")
+    return kc, vc

@@ -338,3 +338,73 @@ int oracle_gather_decode(const oracle_problem* p, const uint8_t* cache,
   }
   return ORACLE_OK;
 }
+
+/* ------------------------------------------------------------------ writer */
+
+/* Nearest e4m3fn value by brute force over the non-negative finite codes
+ * (ascending), ties to the code with the even mantissa; beyond 448 the nearest
+ * is 448 itself, which is the saturation. */
+static int encode_e4m3(float q) {
+  if (isnan(q)) return 0x7F;
+  const double a = fabs((double)q);
+  int best = 0;
+  double best_d = INFINITY;
+  for (int c = 0; c <= 0x7E; ++c) {
+    const double d = fabs(decode_e4m3((uint8_t)c) - a);
+    if (d < best_d || (d == best_d && (c & 1) == 0)) {
+      best = c;
+      best_d = d;
+    }
+  }
+  return (signbit(q) ? 0x80 : 0) | best;
+}
+
+int oracle_quantise(int kv_dtype, float x, float s) {
+  const float q = x / s; /* IEEE single precision (no contraction, no fast math) */
+  if (kv_dtype == ORACLE_KV_FP8_E4M3) return encode_e4m3(q);
+  if (isnan(q)) return 0;
+  const int lo = kv_dtype == ORACLE_KV_INT4 ? -8 : -127;
+  const int hi = kv_dtype == ORACLE_KV_INT4 ? 7 : 127;
+  const float r = rintf(q); /* nearest, ties to even (default rounding mode) */
+  if (r < (float)lo) return lo;
+  if (r > (float)hi) return hi;
+  return (int)r;
+}
+
+static void store_code(const oracle_problem* p, uint8_t* row, int d, int code) {
+  if (p->kv_dtype == ORACLE_KV_INT4) {
+    /* channel 2j low nibble, 2j+1 high nibble of byte j */
+    const uint8_t nib = (uint8_t)(code & 0xF);
+    if (d % 2 == 0)
+      row[d / 2] = (uint8_t)((row[d / 2] & 0xF0) | nib);
+    else
+      row[d / 2] = (uint8_t)((row[d / 2] & 0x0F) | (nib << 4));
+  } else {
+    row[d] = (uint8_t)code;
+  }
+}
+
+int oracle_append(const oracle_problem* p, const double* k_new, const double* v_new,
+                  const float* k_scale, const float* v_scale, const int32_t* block_table,
+                  const int32_t* seqlens_k, const int32_t* cu_seqlens_q, uint8_t* k_cache,
+                  uint8_t* v_cache) {
+  if (check_problem(p, seqlens_k, cu_seqlens_q) != ORACLE_OK) return ORACLE_EINVAL;
+  if (check_block_table(p, block_table, seqlens_k) != ORACLE_OK) return ORACLE_EINVAL;
+  const int Hk = p->kv_num_heads, D = p->head_size;
+  for (int b = 0; b < p->batch; ++b) {
+    const int q0 = cu_seqlens_q[b], qb = cu_seqlens_q[b + 1] - q0, Lb = seqlens_k[b];
+    for (int i = 0; i < qb; ++i) {
+      const int t = (Lb - qb) + i; /* absolute position of new token i */
+      for (int kv = 0; kv < Hk; ++kv) {
+        uint8_t* krow = (uint8_t*)cache_row(p, k_cache, block_table, b, t, kv);
+        uint8_t* vrow = (uint8_t*)cache_row(p, v_cache, block_table, b, t, kv);
+        const int64_t src = ((int64_t)(q0 + i) * Hk + kv) * D;
+        for (int d = 0; d < D; ++d) {
+          store_code(p, krow, d, oracle_quantise(p->kv_dtype, (float)k_new[src + d], k_scale[kv * D + d]));
+          store_code(p, vrow, d, oracle_quantise(p->kv_dtype, (float)v_new[src + d], v_scale[kv * D + d]));
+        }
+      }
+    }
+  }
+  return ORACLE_OK;
+}

@@ -120,6 +120,36 @@ int oracle_paged_attn_partial(const oracle_problem* p, const double* q, const ui
 int oracle_lse_combine(int n_splits, int64_t rows, int head_size, const double* o_parts,
                        const double* lse_parts, double* out);
 
+/* Cache code of one new value x under per-channel scale s, for the
+ * quantise-and-append writer that fills the cache the attention reads (INT4
+ * paged-KV page, Code analysis 2: the cache holds per-channel symmetric codes,
+ * value = scale x code).  The code is decided in IEEE single precision, the
+ * writer's own arithmetic: q = (float)x / s, then
+ *   INT8: nearest integer to q (ties to even), clamped to [-127, 127];
+ *   INT4: the same, clamped to [-8, 7] (the two's complement nibble);
+ *   FP8 : the OCP e4m3fn value nearest to q (ties to the even mantissa),
+ *         magnitudes past 448 saturated to 448; the sign of q is kept on 0.
+ * A NaN quotient gives code 0 (integer caches) or 0x7F (FP8).  Readings (the
+ * pages give the format, not the rounding): round to nearest even, symmetric
+ * INT8 range, saturation.  Returns the signed code (INT8 / INT4) or the byte
+ * (FP8).  Pinned by: exact codes at power-of-two scales, ties, saturation,
+ * the decode table round trip, torch's e4m3fn cast. */
+int oracle_quantise(int kv_dtype, float x, float s);
+
+/* Quantise-and-append: the new K and V rows of every sequence ([T_q, Hk, D]
+ * exact values, packed by cu_seqlens_q) are quantised with oracle_quantise
+ * under k_scale / v_scale [Hk, D] and written at cache slot
+ * block_table[b, t / bs] * bs + t % bs of absolute position t = L_b - q_b + i
+ * for new token i (the cache layout of the INT4 paged-KV page, Code analysis
+ * 2; INT4 channel 2j in the low nibble of byte j).  Every other cache byte is
+ * left as it was.  Contract violations (lengths, block ids) write nothing and
+ * return ORACLE_EINVAL.  Pinned by: placement into a sentinel cache, decode of
+ * the written rows, untouched bytes. */
+int oracle_append(const oracle_problem* p, const double* k_new, const double* v_new,
+                  const float* k_scale, const float* v_scale, const int32_t* block_table,
+                  const int32_t* seqlens_k, const int32_t* cu_seqlens_q, uint8_t* k_cache,
+                  uint8_t* v_cache);
+
 /* Keys of sequence b, dequantised and gathered into contiguous rows:
  * dst[t, d] = decode(cache[block_table[b, t / bs], t % bs, kv, :], d) for
  * t < seqlens_k[b], WITHOUT the per-channel scale (exact small values).

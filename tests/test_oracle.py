@@ -297,3 +297,128 @@ def test_stored_tiny_int8_output_reproduces():
     out = oracle.paged_attn(workloads.oracle_view(w))
     ref = np.loadtxt(os.path.join(GOLDEN, "c1_tiny_int8_oracle.txt")).reshape(out.shape)
     np.testing.assert_allclose(out, ref, rtol=1e-15, atol=0)
+
+
+# ---------------------------------------------------------------- cache writer
+
+
+def test_quantise_exact_codes_at_power_of_two_scales():
+    """x = code * s with s a power of two is exact in fp32: the code comes back,
+    and decoding it times s gives x again (symmetric per-channel format)."""
+    for kv, lo, hi in ((KV_INT8, -127, 127), (KV_INT4, -8, 7)):
+        for s in (2.0 ** -7, 0.5, 1.0, 8.0):
+            for c in range(lo, hi + 1):
+                assert oracle.quantise(kv, c * s, s) == c
+
+
+def test_quantise_ties_round_to_even_and_saturate():
+    s = 0.25
+    for kv in (KV_INT8, KV_INT4):
+        # 0.5, 1.5, 2.5, -0.5, -1.5, -2.5 steps: halves go to the even neighbour
+        assert [oracle.quantise(kv, (c + 0.5) * s, s) for c in (0, 1, 2, -1, -2, -3)] == \
+            [0, 2, 2, 0, -2, -2]
+        assert oracle.quantise(kv, 0.49 * s, s) == 0
+        assert oracle.quantise(kv, 0.51 * s, s) == 1
+    assert oracle.quantise(KV_INT8, 1e6, s) == 127 and oracle.quantise(KV_INT8, -1e6, s) == -127
+    assert oracle.quantise(KV_INT4, 1e6, s) == 7 and oracle.quantise(KV_INT4, -1e6, s) == -8
+    assert oracle.quantise(KV_INT8, float("inf"), s) == 127
+    assert oracle.quantise(KV_INT8, float("nan"), s) == 0
+
+
+def test_quantise_e4m3_round_trips_every_code():
+    """encode(decode(c)) == c for every non-NaN code (the decode table is pinned
+    by the printed code points and torch); 0x80 is the signed zero."""
+    for c in range(256):
+        if (c & 0x7F) == 0x7F:
+            continue
+        v = oracle.decode_row(KV_FP8_E4M3, np.array([c], dtype=np.uint8), 1)[0]
+        assert oracle.quantise(KV_FP8_E4M3, float(v), 1.0) == c, hex(c)
+    assert oracle.quantise(KV_FP8_E4M3, float("nan"), 1.0) == 0x7F
+    assert oracle.quantise(KV_FP8_E4M3, 1e9, 1.0) == 0x7E      # saturates at 448
+    assert oracle.quantise(KV_FP8_E4M3, -1e9, 1.0) == 0xFE
+    assert oracle.quantise(KV_FP8_E4M3, 1.0625, 1.0) == 0x38    # tie 1 | 1.125 -> even
+    assert oracle.quantise(KV_FP8_E4M3, 1.1875, 1.0) == 0x3A    # tie 1.125 | 1.25 -> even
+
+
+def test_quantise_e4m3_matches_torch_cast_in_range():
+    """Inside the finite range the writer's FP8 code is torch's round-to-nearest-
+    even float32 -> float8_e4m3fn cast of the fp32 quotient."""
+    rng = np.random.default_rng(5)
+    x = np.concatenate([rng.standard_normal(4000) * 40, rng.standard_normal(2000) * 0.01,
+                        rng.uniform(-440, 440, 2000)]).astype(np.float32)
+    s = np.float32(1.0)
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.quantise(KV_FP8_E4M3, float(v), float(s)) for v in x], dtype=np.uint8)
+    np.testing.assert_array_equal(got, want)
+
+
+def _append_case(kv, rng, lens, q_lens, bs=16, Hk=2, D=16):
+    prob, _ = paged_problem(rng, kv_dtype=kv, lens=lens, q_lens=q_lens, H=2 * Hk, Hk=Hk, D=D,
+                            bs=bs)
+    T = int(prob["cu_seqlens_q"][-1])
+    k_new = rng.standard_normal((T, Hk, D)) * 3.0
+    v_new = rng.standard_normal((T, Hk, D)) * 3.0
+    if kv == KV_FP8_E4M3:
+        k_new, v_new = k_new * 40.0, v_new * 40.0
+    # the new rows arrive as fp16: their exact values
+    k_new = k_new.astype(np.float16).astype(np.float64)
+    v_new = v_new.astype(np.float16).astype(np.float64)
+    prob["k_scale"] = rng.uniform(0.01, 0.1, size=(Hk, D)).astype(np.float32)
+    prob["v_scale"] = rng.uniform(0.01, 0.1, size=(Hk, D)).astype(np.float32)
+    return prob, k_new, v_new
+
+
+@pytest.mark.parametrize("kv", ALL_KV)
+def test_append_places_rows_at_their_slots_only(kv):
+    """Placement: exactly the bytes of the new tokens' rows change; decoding them
+    gives the codes of the new values; every other byte keeps its old value."""
+    rng = np.random.default_rng(61 + kv)
+    lens, ql = [5, 40, 17, 3], [2, 17, 0, 3]  # crosses block boundaries; one empty sequence
+    prob, k_new, v_new = _append_case(kv, rng, lens, ql)
+    kc, vc = oracle.append(prob, k_new, v_new)
+    bs, Hk, D = prob["block_size"], prob["kv_num_heads"], prob["head_size"]
+    changed_k = np.zeros(kc.shape[:3], dtype=bool)
+    cu = prob["cu_seqlens_q"]
+    for b in range(len(lens)):
+        qb = int(cu[b + 1] - cu[b])
+        for i in range(qb):
+            t = lens[b] - qb + i
+            phys, slot = prob["block_table"][b, t // bs], t % bs
+            changed_k[phys, slot, :] = True
+            for kvh in range(Hk):
+                for new, cache, sc in ((k_new, kc, prob["k_scale"]), (v_new, vc, prob["v_scale"])):
+                    got = oracle.decode_row(kv, cache[phys, slot, kvh], D)
+                    for d in range(D):
+                        code = oracle.quantise(kv, new[cu[b] + i, kvh, d], sc[kvh, d])
+                        want = oracle.decode_row(kv, np.array([code & 0xFF], np.uint8), 1)[0] \
+                            if kv == KV_FP8_E4M3 else code
+                        if np.isnan(want):
+                            assert np.isnan(got[d])
+                        else:
+                            assert got[d] == want
+    np.testing.assert_array_equal(kc[~changed_k], prob["k_cache"][~changed_k])
+    np.testing.assert_array_equal(vc[~changed_k], prob["v_cache"][~changed_k])
+
+
+def test_append_dequant_error_is_half_a_step():
+    """In range, |s * code - x| <= s / 2 for the integer caches (nearest code)."""
+    rng = np.random.default_rng(67)
+    for kv in (KV_INT8, KV_INT4):
+        prob, k_new, v_new = _append_case(kv, rng, [30], [30])
+        k_new = np.clip(k_new, -0.05, 0.05)  # inside the code range at these scales
+        kc, _ = oracle.append(prob, k_new, v_new)
+        bs, D = prob["block_size"], prob["head_size"]
+        for t in range(30):
+            phys, slot = prob["block_table"][0, t // bs], t % bs
+            for kvh in range(prob["kv_num_heads"]):
+                deq = oracle.decode_row(kv, kc[phys, slot, kvh], D) * prob["k_scale"][kvh]
+                assert np.all(np.abs(deq - k_new[t, kvh]) <= prob["k_scale"][kvh] / 2 * (1 + 1e-6))
+
+
+def test_append_rejects_bad_block_ids():
+    rng = np.random.default_rng(71)
+    prob, k_new, v_new = _append_case(KV_INT8, rng, [20], [4])
+    prob["block_table"] = prob["block_table"].copy()
+    prob["block_table"][0, 1] = prob["num_blocks"]  # the page of the new tokens
+    with pytest.raises(ValueError):
+        oracle.append(prob, k_new, v_new)

@@ -5,7 +5,9 @@ source (never in the committed file), builds it, and runs the pin suite in
 tests/test_oracle.py against the broken library.  The pins must catch every
 mistake: a dropped scale, a swapped nibble, a wrong exponent bias, a wrong
 head map, an off-by-one causal limit, a transposed cache index, a flipped
-softmax sign, a wrong combine weight, a wrong fold direction.
+softmax sign, a wrong combine weight, a wrong fold direction; and in the
+cache writer a wrong position, a swapped nibble, truncation instead of
+rounding, a wrong INT8 range and ties to the odd e4m3 code.
 """
 import os
 import shutil
@@ -38,6 +40,12 @@ MUTANTS = {
                        "const double w = exp(lse_parts[sp * rows + r] - mx);"),
     "fold_direction": ("ldexp(k_scale[kv * D + d], -e)", "ldexp(k_scale[kv * D + d], e)"),
     "default_scale": ("1.0 / sqrt((double)p->head_size)", "1.0 / (double)p->head_size"),
+    "append_position": ("const int t = (Lb - qb) + i;", "const int t = i;"),
+    "append_nibble": ("if (d % 2 == 0)\n      row[d / 2] = (uint8_t)((row[d / 2] & 0xF0) | nib);",
+                      "if (d % 2 == 1)\n      row[d / 2] = (uint8_t)((row[d / 2] & 0xF0) | nib);"),
+    "quantise_truncates": ("const float r = rintf(q);", "const float r = truncf(q);"),
+    "quantise_int8_range": ("? -8 : -127;", "? -8 : -128;"),
+    "e4m3_tie_odd": ("(d == best_d && (c & 1) == 0)", "(d == best_d && (c & 1) == 1)"),
 }
 
 
