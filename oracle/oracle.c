@@ -346,6 +346,7 @@ int oracle_gather_decode(const oracle_problem* p, const uint8_t* cache,
  * is 448 itself, which is the saturation. */
 static int encode_e4m3(float q) {
   if (isnan(q)) return 0x7F;
+  if (isinf(q)) return (signbit(q) ? 0x80 : 0) | 0x7E; /* saturation (no infinity code) */
   const double a = fabs((double)q);
   int best = 0;
   double best_d = INFINITY;

@@ -336,6 +336,8 @@ def test_quantise_e4m3_round_trips_every_code():
     assert oracle.quantise(KV_FP8_E4M3, float("nan"), 1.0) == 0x7F
     assert oracle.quantise(KV_FP8_E4M3, 1e9, 1.0) == 0x7E      # saturates at 448
     assert oracle.quantise(KV_FP8_E4M3, -1e9, 1.0) == 0xFE
+    assert oracle.quantise(KV_FP8_E4M3, float("inf"), 1.0) == 0x7E
+    assert oracle.quantise(KV_FP8_E4M3, float("-inf"), 1.0) == 0xFE
     assert oracle.quantise(KV_FP8_E4M3, 1.0625, 1.0) == 0x38    # tie 1 | 1.125 -> even
     assert oracle.quantise(KV_FP8_E4M3, 1.1875, 1.0) == 0x3A    # tie 1.125 | 1.25 -> even
 
