@@ -342,6 +342,69 @@ def measure(name: str, steps: int, warmup: int, dev: str, flush_buf, with_e2e: b
     return res
 
 
+# Quantise-and-append (the cache writer that precedes the attention call):
+# (name, description, new tokens, sequences, Hk, D, block_size, kv dtype, bf16 input)
+APPEND = [("append_prefill_32k_int8", "append of a 32768-token prompt: Hk=8 D=128 bs=16 INT8, "
+           "bf16 K/V in", 32768, 1, 8, 128, 16, workloads.KV_INT8, True),
+          ("append_decode_int4", "decode-step append: 16 sequences x 1 token, Hk=8 D=128 bs=16 "
+           "INT4, fp16 K/V in", 16, 16, 8, 128, 16, workloads.KV_INT4, False)]
+
+
+def measure_append(spec, steps: int, warmup: int, dev: str, flush_buf):
+    """Device time of paged_kv_append (CUDA events on the launching stream)."""
+    import paged_quantized_kv_attention_b200 as pa
+    name, desc, T, B, Hk, D, bs, kv, bf16 = spec
+    rng = np.random.default_rng(2024)
+    per = T // B
+    cu = np.arange(0, T + 1, per, dtype=np.int32)
+    sk = np.full(B, 4096 if B > 1 else T, dtype=np.int32)  # decode: 4095 past keys each
+    nblk = int(-(-sk.max() // bs))
+    pool = B * nblk * 2
+    bt = rng.permutation(pool)[:B * nblk].astype(np.int32).reshape(B, nblk)
+    chs = D // 2 if kv == workloads.KV_INT4 else D
+    dt = torch.bfloat16 if bf16 else torch.float16
+    kc = torch.zeros((pool, bs, Hk, chs), dtype=torch.uint8, device=dev)
+    vc = torch.zeros_like(kc)
+    kn = (torch.randn((T, Hk, D), device=dev) * 3).to(dt)
+    vn = (torch.randn((T, Hk, D), device=dev) * 3).to(dt)
+    ks = torch.from_numpy(rng.uniform(0.01, 0.1, (Hk, D)).astype(np.float32)).to(dev)
+    vs = torch.from_numpy(rng.uniform(0.01, 0.1, (Hk, D)).astype(np.float32)).to(dev)
+    p = pa.make_params(batch=B, num_heads=Hk, kv_num_heads=Hk, head_size=D, block_size=bs,
+                       num_blocks=pool, max_blocks_per_seq=nblk, kv_dtype=kv,
+                       q_dtype=1 if bf16 else 0, out_dtype=1 if bf16 else 0)
+    nb = pa.paged_attn_plan(cu, sk, p)
+    ws = torch.zeros(max(nb, 256), dtype=torch.uint8, device=dev)
+    p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
+    args = (kn, vn, kc, vc, ks, vs, torch.from_numpy(bt).to(dev), torch.from_numpy(sk).to(dev),
+            torch.from_numpy(cu).to(dev))
+    big = 2 * T * Hk * D * 2 > L2_BYTES  # the new rows alone stream through L2 every step
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        pa.paged_kv_append(*args, p, stream)
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(steps):
+        if not big:
+            flush_buf.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        pa.paged_kv_append(*args, p, stream)
+        e1.record(stream)
+        e1.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    st, bits = pa.paged_attn_read_device_error(ws)
+    k_ms = statistics.median(ms)
+    nbytes = (2 * T * Hk * D * 2 + 2 * T * Hk * chs + 2 * Hk * D * 4 + T * 4 + 2 * (B + 1) * 4)
+    peak, kind = measured_peaks()
+    gbs = nbytes / (k_ms * 1e-3) / 1e9
+    return {"desc": desc, "us_per_call": round(k_ms * 1e3, 3), "gbs": round(gbs, 1),
+            "frac_of_measured_peak" if kind == "measured" else "frac_of_fallback_peak":
+                round(gbs / peak, 4),
+            "algorithmic_bytes": nbytes, "device_error_bits": bits,
+            "l2": "inputs larger than L2" if big else "flushed before every call (256 MB write)",
+            "kernel": "pa_append_kernel"}
+
+
 def summary_of(name, r):
     return {"workload": name, "desc": workloads.DESCRIPTIONS[name],
             "gbs": round(r["value"], 1), "us_per_call": round(r["call_ms"] * 1e3, 2),
@@ -392,6 +455,8 @@ def run_ours(args):
             rr = measure(name, max(3, min(args.steps, 20)), args.warmup, dev, flush,
                          with_e2e=False)
             extra[name] = summary_of(name, rr)
+        for spec in APPEND:
+            extra[spec[0]] = measure_append(spec, max(5, min(args.steps, 20)), 3, dev, flush)
     if rank != 0:
         if dist is not None:
             dist.destroy_process_group()

@@ -124,14 +124,17 @@ int oracle_lse_combine(int n_splits, int64_t rows, int head_size, const double* 
  * quantise-and-append writer that fills the cache the attention reads (INT4
  * paged-KV page, Code analysis 2: the cache holds per-channel symmetric codes,
  * value = scale x code).  The code is decided in IEEE single precision, the
- * writer's own arithmetic: q = (float)x / s, then
+ * writer's own arithmetic: q = (float)x * inv with inv = 1 / s rounded to fp32
+ * (a multiply by the per-channel inverse scale), then
  *   INT8: nearest integer to q (ties to even), clamped to [-127, 127];
  *   INT4: the same, clamped to [-8, 7] (the two's complement nibble);
  *   FP8 : the OCP e4m3fn value nearest to q (ties to the even mantissa),
  *         magnitudes past 448 saturated to 448; the sign of q is kept on 0.
  * A NaN quotient gives code 0 (integer caches) or 0x7F (FP8).  Readings (the
  * pages give the format, not the rounding): round to nearest even, symmetric
- * INT8 range, saturation.  Returns the signed code (INT8 / INT4) or the byte
+ * INT8 range, saturation, the inverse-scale multiply (one rounding of 1/s,
+ * one of the product; a correctly rounded x / s would differ from it only at
+ * rare rounding boundaries).  Returns the signed code (INT8 / INT4) or the byte
  * (FP8).  Pinned by: exact codes at power-of-two scales, ties, saturation,
  * the decode table round trip, torch's e4m3fn cast. */
 int oracle_quantise(int kv_dtype, float x, float s);

@@ -195,6 +195,37 @@ def test_forward_checks_arguments_before_any_launch():
     assert ei.value.status == pa.PA_ERR_INVALID_ARG
 
 
+def test_append_checks_arguments_before_any_launch():
+    cu = np.array([0, 3], dtype=np.int32)
+    p = _params(batch=1)
+    pa.paged_attn_plan(cu, np.array([40]), p)
+    buf = np.zeros(4096, dtype=np.uint8)
+    al = buf[(-buf.ctypes.data) % 256:]  # 256-aligned host memory, never dereferenced here
+    args = [al] * 9
+    # a NULL pointer
+    p.workspace, p.workspace_bytes = al.ctypes.data, 256
+    bad = list(args)
+    bad[4] = None
+    with pytest.raises(pa.PagedAttnError) as ei:
+        pa.paged_kv_append(*bad, p, stream=0)
+    assert ei.value.status == pa.PA_ERR_INVALID_ARG
+    # misaligned new rows
+    bad = list(args)
+    bad[0] = al[4:]
+    with pytest.raises(pa.PagedAttnError) as ei:
+        pa.paged_kv_append(*bad, p, stream=0)
+    assert ei.value.status == pa.PA_ERR_INVALID_ARG
+    # no workspace for the error word
+    p.workspace, p.workspace_bytes = None, 0
+    with pytest.raises(pa.PagedAttnError) as ei:
+        pa.paged_kv_append(*args, p, stream=0)
+    assert ei.value.status == pa.PA_ERR_WORKSPACE
+    # no new tokens: nothing to do, nothing launched
+    p0 = _params(batch=1)
+    pa.paged_attn_plan(np.array([0, 0], dtype=np.int32), np.array([40]), p0)
+    pa.paged_kv_append(*args, p0, stream=0)
+
+
 def test_codec_entry_points_check_arguments():
     with pytest.raises(pa.PagedAttnError):
         pa.paged_kv_pack_int4(None, None, 4, 128, stream=0)
