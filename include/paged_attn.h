@@ -222,6 +222,39 @@ pa_status paged_kv_pack_int4(const int8_t* src, uint8_t* dst, int64_t rows, int 
 pa_status paged_kv_unpack_int4(const uint8_t* src, int8_t* dst, int64_t rows, int head_size,
                                void* stream);
 
+/* Quantise-and-append: the cache write that precedes the attention call (the
+ * INT4 paged-KV page, Code analysis 2-3: per-channel symmetric codes,
+ * value = scale x code, in the [num_blocks, block_size, Hk, chs] cache).
+ *
+ * For every sequence b and new token i < q_b (q_b from cu_seqlens_q), at
+ * absolute position t = seqlens_k[b] - q_b + i, the K and V rows of that token
+ * (k_new / v_new, [total_q, Hk, head_size] in params->q_dtype, packed by
+ * cu_seqlens_q like q) are stored at cache slot block_table[b, t / block_size]
+ * * block_size + t % block_size, head kv.  Channel d's code is decided in IEEE
+ * single precision from q = x / scale[kv, d] (correctly rounded division):
+ *   INT8: nearest integer (ties to even) clamped to [-127, 127];
+ *   INT4: the same clamped to [-8, 7], channel 2j in the low nibble of byte j;
+ *   FP8 : round-to-nearest-even e4m3fn, saturating at +-448.
+ * A NaN quotient stores 0 (integer caches) or 0x7F (FP8).  No other cache byte
+ * is written.
+ *
+ * params: the plan of the same call (paged_attn_plan sets total_q); batch,
+ * kv_num_heads, head_size, block_size, num_blocks, max_blocks_per_seq,
+ * kv_dtype and q_dtype are read, and params->workspace (device, 256-byte
+ * aligned, >= 256 bytes) holds the device error word of byte 0 as for
+ * paged_attn_forward.  All array pointers are device pointers; k_new, v_new,
+ * the scales and the caches must be 16-byte aligned.  The caller owns every
+ * buffer.  A row whose sequence lengths are invalid or whose block id lies
+ * outside [0, num_blocks) is not written and sets PA_DEVERR_BAD_LENGTH /
+ * PA_DEVERR_BAD_BLOCK in the error word (read with
+ * paged_attn_read_device_error).  Host-checked violations return an error
+ * status with nothing launched; total_q == 0 returns PA_OK.  Asynchronous on
+ * `stream`. */
+pa_status paged_kv_append(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                          const float* k_scale, const float* v_scale, const int32_t* block_table,
+                          const int32_t* seqlens_k, const int32_t* cu_seqlens_q,
+                          const paged_attn_params* params, void* stream);
+
 /* Test hook: gather the keys (or values) of sequence b, KV head kv through the
  * block table, decode them with the attention kernel's conversion routines and
  * store the exact unscaled codes as fp16 (dst_dtype PA_F16) or bf16 (PA_BF16),

@@ -26,8 +26,8 @@ PA_NOALLOC_MAX_WORKSPACE_BYTES = 16 << 20
 EXPORTED = ["paged_attn_plan", "paged_attn_forward", "paged_attn_forward_noalloc",
             "paged_attn_workspace_init",
             "paged_attn_read_device_error", "paged_kv_pack_int4", "paged_kv_unpack_int4",
-            "paged_kv_gather_decode", "paged_attn_stream_read", "paged_attn_last_error",
-            "paged_attn_version"]
+            "paged_kv_gather_decode", "paged_kv_append", "paged_attn_stream_read",
+            "paged_attn_last_error", "paged_attn_version"]
 
 
 class PagedAttnError(RuntimeError):
@@ -73,6 +73,7 @@ def lib() -> ctypes.CDLL:
         L.paged_kv_pack_int4.argtypes = [P, P, ctypes.c_int64, I, P]
         L.paged_kv_unpack_int4.argtypes = [P, P, ctypes.c_int64, I, P]
         L.paged_kv_gather_decode.argtypes = [P, P, PP, I, I, I, I, P, P]
+        L.paged_kv_append.argtypes = [P] * 9 + [PP, P]
         L.paged_attn_stream_read.argtypes = [P, S, P, P]
         L.paged_attn_last_error.restype = ctypes.c_char_p
         L.paged_attn_version.restype = ctypes.c_char_p
@@ -168,6 +169,15 @@ def paged_kv_gather_decode(cache, block_table, params: paged_attn_params, b: int
                            len_b: int, dst_dtype: int, dst, stream=None):
     _check(lib().paged_kv_gather_decode(_ptr(cache), _ptr(block_table), ctypes.byref(params), b,
                                         kv, len_b, dst_dtype, _ptr(dst), _stream(stream)))
+
+
+def paged_kv_append(k_new, v_new, k_cache, v_cache, k_scale, v_scale, block_table, seqlens_k,
+                    cu_seqlens_q, params: paged_attn_params, stream=None):
+    """Quantise the new tokens' K/V rows ([total_q, Hk, D], params.q_dtype) into
+    the caches at their slots (see paged_kv_append in paged_attn.h)."""
+    _check(lib().paged_kv_append(_ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+                                 _ptr(k_scale), _ptr(v_scale), _ptr(block_table), _ptr(seqlens_k),
+                                 _ptr(cu_seqlens_q), ctypes.byref(params), _stream(stream)))
 
 
 def paged_attn_stream_read(src, nbytes: int, sink, stream=None):

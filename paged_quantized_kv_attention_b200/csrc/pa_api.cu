@@ -468,6 +468,48 @@ pa_status paged_kv_gather_decode(const void* cache, const int32_t* block_table,
   return e == cudaSuccess ? ok() : cuda_status(e, "gather_decode launch");
 }
 
+pa_status paged_kv_append(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                          const float* k_scale, const float* v_scale, const int32_t* block_table,
+                          const int32_t* seqlens_k, const int32_t* cu_seqlens_q,
+                          const paged_attn_params* p, void* stream) {
+  pa_status st = check_problem(p);
+  if (st != PA_OK) return st;
+  if (p->total_q < 0) return fail(PA_ERR_INVALID_ARG, "total_q %d < 0 (call paged_attn_plan)", p->total_q);
+  if (p->total_q == 0 || p->batch == 0) return ok();
+  if (!k_new || !v_new || !k_cache || !v_cache || !k_scale || !v_scale || !block_table ||
+      !seqlens_k || !cu_seqlens_q)
+    return fail(PA_ERR_INVALID_ARG, "NULL pointer argument");
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_scale, 16) ||
+      !aligned(v_scale, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16))
+    return fail(PA_ERR_INVALID_ARG, "new rows, scales and caches must be 16-byte aligned");
+  if (p->workspace == nullptr || p->workspace_bytes < kHeaderBytes ||
+      !aligned(p->workspace, 256))
+    return fail(PA_ERR_WORKSPACE, "a 256-byte aligned workspace of >= 256 bytes holds the error word");
+  if (static_cast<int64_t>(p->kv_num_heads) * p->head_size * 8 > 200 * 1024)
+    return fail(PA_ERR_UNSUPPORTED, "kv_num_heads x head_size too large for the writer's "
+                "shared-memory inverse scales");
+  pa::AppendArgs a;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
+  a.block_table = block_table;
+  a.seqlens_k = seqlens_k;
+  a.cu_seqlens_q = cu_seqlens_q;
+  a.err = static_cast<uint32_t*>(p->workspace);
+  a.batch = p->batch;
+  a.Hk = p->kv_num_heads;
+  a.maxb = p->max_blocks_per_seq;
+  a.num_blocks = p->num_blocks;
+  a.block_size = p->block_size;
+  a.total_q = p->total_q;
+  a.in_bf16 = p->q_dtype == PA_BF16;
+  cudaError_t e = pa::launch_append(p->kv_dtype, p->head_size, a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ok() : cuda_status(e, "append launch");
+}
+
 pa_status paged_attn_stream_read(const void* src, size_t bytes, void* sink, void* stream) {
   if (!src || !sink) return fail(PA_ERR_INVALID_ARG, "src/sink is NULL");
   if (bytes % 16 != 0 || !aligned(src, 16) || !aligned(sink, 16))

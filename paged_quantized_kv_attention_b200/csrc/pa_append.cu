@@ -1,0 +1,182 @@
+// pa_append.cu -- quantise-and-append: the cache write that precedes the
+// attention call.  The new K and V rows of every sequence's new tokens are
+// turned into per-channel symmetric codes (value = scale x code, the cache
+// format of the INT4 paged-KV page, onnxruntime PR 32515, Code analysis 2-3)
+// and stored at the slot the block table gives their absolute position.
+//
+// The code of a value is decided in IEEE single precision: q = x * inv, inv the
+// fp32-rounded inverse of the channel's scale, then INT8: nearest integer, ties
+// to even, clamped to
+// [-127, 127]; INT4: the same clamped to [-8, 7], channel 2j in the low nibble of
+// byte j; FP8: round-to-nearest-even e4m3fn, saturating at +-448.  A NaN quotient
+// stores 0 (integer caches) or 0x7F (FP8).
+//
+// HBM-bound and elementwise: a warp takes one new token's K or V rows; lane l
+// handles 8-channel groups l, l + 32, ... of the token's Hk x D values (16 bytes
+// of fp16/bf16 in, 8 or 4 bytes out), so both the reads and the row writes of a
+// token (its heads are contiguous in the cache slot) are contiguous.
+#include <cuda_fp8.h>
+
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+
+__device__ __forceinline__ float bits_to_float(uint32_t h, bool bf16) {
+  return bf16 ? __uint_as_float(h << 16)
+              : __half2float(__ushort_as_half(static_cast<unsigned short>(h)));
+}
+
+// x times the inverse scale inv = 1 / s (rounded to fp32 once per channel).
+template <int KV>
+__device__ __forceinline__ uint32_t code_of(float x, float inv) {
+  const float q = __fmul_rn(x, inv);
+  if constexpr (KV == PA_KV_FP8_E4M3) {
+    if (q != q) return 0x7Fu;
+    return static_cast<uint32_t>(__nv_cvt_float_to_fp8(q, __NV_SATFINITE, __NV_E4M3)) & 0xFFu;
+  } else {
+    if (q != q) return 0u;
+    constexpr float lo = KV == PA_KV_INT4 ? -8.f : -127.f;
+    constexpr float hi = KV == PA_KV_INT4 ? 7.f : 127.f;
+    const float r = fminf(fmaxf(rintf(q), lo), hi);
+    return static_cast<uint32_t>(static_cast<int>(r)) & (KV == PA_KV_INT4 ? 0xFu : 0xFFu);
+  }
+}
+
+// Quantise 8 channels (16 input bytes) into their packed codes: 4 bytes (INT4)
+// or 8 bytes (INT8, FP8) in the low bits of out.
+template <int KV>
+__device__ __forceinline__ uint2 codes8(uint4 raw, float4 s0, float4 s1, bool bf16) {
+  const float s[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};  // inverse scales
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+  uint32_t c[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e)
+    c[e] = code_of<KV>(bits_to_float((w[e >> 1] >> (16 * (e & 1))) & 0xFFFFu, bf16), s[e]);
+  if constexpr (KV == PA_KV_INT4) {
+    uint32_t out = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) out |= (c[2 * j] | (c[2 * j + 1] << 4)) << (8 * j);
+    return make_uint2(out, 0u);
+  } else {
+    return make_uint2(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24),
+                      c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24));
+  }
+}
+
+// One warp per new token, grid-striding over total_q: the warp decodes the
+// token's sequence, position and page once, then its lanes walk the token's
+// Hk x D/8 channel groups of K and of V together (16 input bytes each,
+// contiguous across the lanes; all of a lane's loads go out before any code is
+// computed).
+template <int KV, int D>
+__global__ void __launch_bounds__(256) pa_append_kernel(AppendArgs a) {
+  constexpr int kGroups = D / 8;
+  constexpr int kChs = KV == PA_KV_INT4 ? D / 2 : D;
+  constexpr int kU = 4;  // groups per lane per pass (of K and of V)
+  // inverse scales of every channel, K then V: [2][Hk][D] fp32
+  extern __shared__ float4 inv_s[];
+  float* inv = reinterpret_cast<float*>(inv_s);
+  for (int i = threadIdx.x; i < a.Hk * D; i += blockDim.x) {
+    inv[i] = __frcp_rn(__ldg(a.k_scale + i));
+    inv[a.Hk * D + i] = __frcp_rn(__ldg(a.v_scale + i));
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int nwarps = static_cast<int>((gridDim.x * blockDim.x) >> 5);
+  const int per_tok = a.Hk * kGroups;
+  for (int tok = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+       tok < a.total_q; tok += nwarps) {
+    // sequence of the token: the last b with cu[b] <= tok (warp-uniform)
+    int lo = 0, hi = a.batch - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (__ldg(a.cu_seqlens_q + mid) <= tok) lo = mid; else hi = mid - 1;
+    }
+    const int b = lo;
+    const int q0 = __ldg(a.cu_seqlens_q + b), qb = __ldg(a.cu_seqlens_q + b + 1) - q0;
+    const int Lb = __ldg(a.seqlens_k + b);
+    if (qb <= 0 || qb > Lb || tok - q0 >= qb ||
+        static_cast<long long>(Lb) > static_cast<long long>(a.maxb) * a.block_size) {
+      if (lane == 0) record_error(a.err, PA_DEVERR_BAD_LENGTH);
+      continue;
+    }
+    const int t = (Lb - qb) + (tok - q0);  // absolute position of the new token
+    const int phys = __ldg(a.block_table + static_cast<size_t>(b) * a.maxb + t / a.block_size);
+    if (phys < 0 || phys >= a.num_blocks) {
+      if (lane == 0) record_error(a.err, PA_DEVERR_BAD_BLOCK);
+      continue;  // the slot is unknown: nothing is written
+    }
+    const int slot = t % a.block_size;
+    const size_t src_off = static_cast<size_t>(tok) * a.Hk * D;
+    const uint4* ksrc = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.k_new) + src_off);
+    const uint4* vsrc = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.v_new) + src_off);
+    const size_t dst_off = (static_cast<size_t>(phys) * a.block_size + slot) * a.Hk * kChs;
+    uint8_t* kdst = static_cast<uint8_t*>(a.k_cache) + dst_off;
+    uint8_t* vdst = static_cast<uint8_t*>(a.v_cache) + dst_off;
+    for (int g0 = 0; g0 < per_tok; g0 += 32 * kU) {
+      uint4 kr[kU], vr[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int gi = g0 + 32 * u + lane;
+        kr[u] = gi < per_tok ? __ldg(ksrc + gi) : make_uint4(0u, 0u, 0u, 0u);
+        vr[u] = gi < per_tok ? __ldg(vsrc + gi) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int gi = g0 + 32 * u + lane;
+        if (gi >= per_tok) break;
+        // channels gi * 8 .. gi * 8 + 7 of the token's Hk x D row set
+        const float4* ki = inv_s + 2 * gi;
+        const float4* vi = inv_s + (a.Hk * D) / 4 + 2 * gi;
+        const uint2 kc = codes8<KV>(kr[u], ki[0], ki[1], a.in_bf16);
+        const uint2 vc = codes8<KV>(vr[u], vi[0], vi[1], a.in_bf16);
+        // group gi is bytes [gi * 8, gi * 8 + 8) of the slot's Hk rows (INT4: 4)
+        if constexpr (KV == PA_KV_INT4) {
+          reinterpret_cast<uint32_t*>(kdst)[gi] = kc.x;
+          reinterpret_cast<uint32_t*>(vdst)[gi] = vc.x;
+        } else {
+          reinterpret_cast<uint2*>(kdst)[gi] = kc;
+          reinterpret_cast<uint2*>(vdst)[gi] = vc;
+        }
+      }
+    }
+  }
+}
+
+template <int KV, int D>
+static cudaError_t launch_append_t(const AppendArgs& a, cudaStream_t stream) {
+  if (a.total_q <= 0) return cudaSuccess;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long tasks = a.total_q;  // one warp per new token, 8 warps per CTA
+  const long long want = (tasks + 7) / 8;
+  const long long cap = static_cast<long long>(sms) * 8;  // 8 CTAs of 8 warps per SM
+  const size_t smem = static_cast<size_t>(a.Hk) * D * 2 * sizeof(float);
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(pa_append_kernel<KV, D>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  pa_append_kernel<KV, D><<<static_cast<unsigned>(want < cap ? want : cap), 256, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append(int kv_dtype, int head_size, const AppendArgs& a, cudaStream_t stream) {
+  const bool d128 = head_size == 128;
+  switch (kv_dtype) {
+    case PA_KV_INT8:
+      return d128 ? launch_append_t<PA_KV_INT8, 128>(a, stream) : launch_append_t<PA_KV_INT8, 64>(a, stream);
+    case PA_KV_INT4:
+      return d128 ? launch_append_t<PA_KV_INT4, 128>(a, stream) : launch_append_t<PA_KV_INT4, 64>(a, stream);
+    case PA_KV_FP8_E4M3:
+      return d128 ? launch_append_t<PA_KV_FP8_E4M3, 128>(a, stream)
+                  : launch_append_t<PA_KV_FP8_E4M3, 64>(a, stream);
+    default:
+      return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace pa

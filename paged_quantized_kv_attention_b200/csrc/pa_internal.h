@@ -60,6 +60,23 @@ __host__ __device__ inline void split_geometry(int nblk, int T, int max_splits, 
 constexpr size_t kWsHeaderBytes = 256;
 constexpr size_t kWsWorkOffset = 64;
 
+// Arguments of the quantise-and-append writer (pa_append.cu).
+struct AppendArgs {
+  const void* k_new;  // [total_q, Hk, D] fp16 / bf16
+  const void* v_new;
+  void* k_cache;      // [num_blocks, block_size, Hk, chs]
+  void* v_cache;
+  const float* k_scale;  // [Hk, D]
+  const float* v_scale;
+  const int32_t* block_table;
+  const int32_t* seqlens_k;
+  const int32_t* cu_seqlens_q;
+  uint32_t* err;      // device error word (workspace byte 0)
+  int batch, Hk, maxb, num_blocks, block_size, total_q;
+  bool in_bf16;
+};
+cudaError_t launch_append(int kv_dtype, int head_size, const AppendArgs& a, cudaStream_t stream);
+
 // Launcher (pa_attention.cu).  rows_per_cta is 4 (decode rows packed with their
 // fp16 residuals), 8 or 16.
 cudaError_t launch_forward(int kv_dtype, int head_size, int block_size, int rows_per_cta,
