@@ -557,9 +557,18 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--writer", action="store_true",
+                    help="time only the quantise-and-append writer workloads (one JSON line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.writer:
+        torch.cuda.set_device(0)
+        flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda:0")
+        print(json.dumps({"writer": {spec[0]: measure_append(spec, args.steps, args.warmup,
+                                                             "cuda:0", flush)
+                                     for spec in APPEND}}))
+        return
     if args.impl == "reference":
         run_reference(args)
     else:
