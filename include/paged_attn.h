@@ -94,7 +94,7 @@ typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
 /* Bits of the device error word (see paged_attn_read_device_error). */
 #define PA_DEVERR_BAD_BLOCK 0x1u   /* block_table entry outside [0, num_blocks) */
 #define PA_DEVERR_TIMEOUT 0x2u     /* an mbarrier wait exceeded its time bound */
-#define PA_DEVERR_BAD_SCALE 0x4u   /* max |k_scale| of a KV head is not finite */
+#define PA_DEVERR_BAD_SCALE 0x4u   /* a K or V scale of a KV head is not finite */
 #define PA_DEVERR_BAD_LENGTH 0x8u  /* device seqlens/cu_seqlens contradict the plan */
 
 typedef struct {
@@ -159,7 +159,13 @@ pa_status paged_attn_plan(const int32_t* cu_seqlens_q_host, const int32_t* seqle
  * launched as the forward kernel's programmatic dependent (it overlaps the
  * forward kernel's tail and waits for its completion).  q, k_scale
  * and v_scale must be 16-byte aligned, the caches 16-byte aligned, out 4-byte
- * aligned.  After a device error the workspace should be re-initialised. */
+ * aligned.  After a device error the workspace should be re-initialised.
+ * Extreme scales (the INT4 paged-KV page's lesson on FLT_MAX scales): K scales
+ * and queries of any finite magnitude, up to FLT_MAX, give finite outputs that
+ * follow the definition (when the logits leave fp32 range the softmax is the
+ * hard maximum it tends to); a NaN or infinite K or V scale sets
+ * PA_DEVERR_BAD_SCALE and the output rows are then undefined.  Outputs whose
+ * true value exceeds the output type's range round to +-infinity. */
 pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_cache,
                              const float* k_scale, const float* v_scale,
                              const int32_t* block_table, const int32_t* seqlens_k,

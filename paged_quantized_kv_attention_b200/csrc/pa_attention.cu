@@ -290,11 +290,15 @@ __device__ __forceinline__ void query_fragments(const FwdArgs& a, const uint8_t*
     }
   }
   float ksmax = 0.f;
+  bool scale_ok = true;  // every K scale of the head finite (a NaN escapes fmaxf)
 #pragma unroll
-  for (int i = 0; i < kN; ++i) ksmax = fmaxf(ksmax, fabsf(sc[i]));
+  for (int i = 0; i < kN; ++i) {
+    ksmax = fmaxf(ksmax, fabsf(sc[i]));
+    scale_ok &= isfinite(sc[i]);
+  }
   ksmax = fmaxf(ksmax, __shfl_xor_sync(kFull, ksmax, 1));
   ksmax = fmaxf(ksmax, __shfl_xor_sync(kFull, ksmax, 2));
-  if (!isfinite(ksmax) && lane == 0) record_error(a.err, PA_DEVERR_BAD_SCALE);
+  if (__any_sync(kFull, !scale_ok) && lane == 0) record_error(a.err, PA_DEVERR_BAD_SCALE);
   int e_kv = 0;
   (void)frexpf(ksmax, &e_kv);
   const float f_kv = ldexpf(1.f, -e_kv);
@@ -318,7 +322,12 @@ __device__ __forceinline__ void query_fragments(const FwdArgs& a, const uint8_t*
     rmax = fmaxf(rmax, __shfl_xor_sync(kFull, rmax, 2));
     int e_q = 0;
     (void)frexpf(rmax, &e_q);
-    crow[nt] = ldexpf(a.sm_scale_log2, e_kv + e_q);
+    // The multiplier is capped at 2^90 (K scales or queries near FLT_MAX would
+    // overflow it): the logits stay below 2^110, and two logits whose products
+    // differ by 2^-31 of the query's digit unit or more still differ by >= 2^59
+    // in log2 units, so the fp32 softmax weights are the same hard maximum the
+    // uncapped values give.
+    crow[nt] = fminf(ldexpf(a.sm_scale_log2, e_kv + e_q), 0x1p90f);
     if constexpr (C::kInt) {
       const float f = ldexpf(1.f, 6 - e_q);
       const int p = g & 1;
@@ -406,6 +415,11 @@ __global__ void __launch_bounds__(64) pa_prep_kernel(const FwdArgs a) {
                       (static_cast<size_t>(q0) * a.H + static_cast<size_t>(h) * a.G) * D * 2;
   query_fragments<KV, D, BS, NT, LP>(a, qh, a.k_scale + static_cast<size_t>(h) * D, row0, nrows,
                                      lane, qf, crow);
+  if (rg == 0) {  // the head's V scales must be finite too (once per sequence and head)
+    bool ok = true;
+    for (int d = lane; d < D; d += 32) ok &= isfinite(__ldg(a.v_scale + static_cast<size_t>(h) * D + d));
+    if (__any_sync(kFull, !ok) && lane == 0) record_error(a.err, PA_DEVERR_BAD_SCALE);
+  }
   uint32_t* fb = a.frag + static_cast<size_t>(u) * C::kUnitWords;
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {

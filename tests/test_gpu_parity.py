@@ -216,6 +216,57 @@ def test_non_finite_k_scale_is_flagged():
     assert bits & pa.PA_DEVERR_BAD_SCALE
 
 
+@pytest.mark.parametrize("which,val", [("k", np.nan), ("v", np.nan), ("v", -np.inf)])
+def test_nan_or_infinite_scale_is_flagged(which, val):
+    """A NaN K scale (which a max over the channels would skip), or a non-finite
+    V scale, sets the defined error bit; nothing faults."""
+    rng = np.random.default_rng(5)
+    prob, _ = paged_problem(rng, kv_dtype=KV_INT4, lens=[40, 70], q_lens=[1, 1], H=8, Hk=2,
+                            D=128, bs=16)
+    w = _as_workload(prob, 0, 0)
+    key = which + "_scale"
+    w[key] = w[key].copy()
+    w[key][1, 77] = val
+    out, p, ws = _gpu.run(w)
+    st, bits = pa.paged_attn_read_device_error(ws)
+    assert bits & pa.PA_DEVERR_BAD_SCALE
+
+
+@pytest.mark.parametrize("kv", ALL_KV)
+@pytest.mark.parametrize("kmag", [3.0e38, 1.0e30, 1.0e-30])
+def test_extreme_k_scales_follow_the_oracle(kv, kmag):
+    """K scales up to FLT_MAX (and down to 1e-30): finite outputs equal to the
+    oracle's (which, for huge scales, is the V row of the largest logit)."""
+    rng = np.random.default_rng(int(np.log10(kmag) + 100) + kv)
+    Hk, D = 2, 128
+    k_scale = (kmag * rng.uniform(0.25, 1.0, size=(Hk, D))).astype(np.float32)
+    prob, _ = paged_problem(rng, kv_dtype=kv, lens=[60, 33, 90], q_lens=[1, 4, 1], H=8, Hk=Hk,
+                            D=D, bs=16, k_scale=k_scale)
+    w = _as_workload(prob, 1, 1)
+    assert np.all(np.isfinite(w["k_scale"]))
+    for split in (-1, 2):
+        out, p, ws = _gpu.run(w, split_blocks=split)
+        st, bits = pa.paged_attn_read_device_error(ws)
+        assert bits == 0
+        got = out.double().cpu().numpy()
+        assert np.all(np.isfinite(got))
+        _check(w, out)
+
+
+def test_queries_near_bf16_max_stay_finite():
+    """bf16 queries of magnitude 1e38 (the multiplier would overflow without its
+    cap): finite outputs equal to the oracle's."""
+    rng = np.random.default_rng(98)
+    prob, _ = paged_problem(rng, kv_dtype=KV_INT8, lens=[50, 20], q_lens=[1, 2], H=8, Hk=2,
+                            D=128, bs=16)
+    w = _as_workload(prob, 1, 1)
+    w["q"] = (w["q"].float().clamp(-3.0, 3.0) * 1.0e38).to(torch.bfloat16)  # |q| <= 3e38
+    assert bool(torch.isfinite(w["q"]).all())
+    out, _, ws = _gpu.run(w)
+    assert pa.paged_attn_read_device_error(ws)[1] == 0
+    _check(w, out)
+
+
 # ------------------------------------------------------------- full sizes, sampled
 
 
