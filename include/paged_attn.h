@@ -138,6 +138,12 @@ typedef struct {
                              cudaEvent_t that paged_attn_forward records on the
                              stream right before and right after the fused
                              attention kernel launch */
+  float* lse_out;         /* optional: NULL, or device [total_q, num_heads] fp32
+                             that receives each row's log-sum-exp of its scaled
+                             logits, log sum_t exp(s_t) (natural log; -inf when the
+                             row sees no key), so that results over disjoint key
+                             sets merge exactly (paged_attn_merge; the GQA GEMV
+                             decode page, Code analysis 2) */
 } paged_attn_params;
 
 /* Host-side planner.  Validates the problem, computes the exact max_query_len
@@ -227,6 +233,19 @@ pa_status paged_kv_pack_int4(const int8_t* src, uint8_t* dst, int64_t rows, int 
                              void* stream);
 pa_status paged_kv_unpack_int4(const uint8_t* src, int8_t* dst, int64_t rows, int head_size,
                                void* stream);
+
+/* Log-sum-exp merge of attention results over disjoint key sets (the flash-
+ * decoding combine of the GQA GEMV decode page, Code analysis 2, across calls:
+ * context parallelism, one key range per GPU).  parts: [n_parts, rows,
+ * head_size] in dtype (PA_F16 / PA_BF16), each part normalised over its own
+ * keys; lse_parts: [n_parts, rows] fp32, natural log, -inf for a part with no
+ * key (as paged_attn_forward's lse_out gives them).  out[r] = sum_p
+ * exp(lse_p[r] - lse[r]) parts[p, r] with lse[r] = log sum_p exp(lse_p[r]),
+ * rounded to dtype; a row with no key in any part gets zeros.  lse_out
+ * (optional, [rows]) receives lse.  1 <= n_parts <= 64; head_size 64 or 128;
+ * device pointers, parts/out 8-byte aligned; async on `stream`. */
+pa_status paged_attn_merge(const void* parts, const float* lse_parts, int n_parts, int64_t rows,
+                           int head_size, int dtype, void* out, float* lse_out, void* stream);
 
 /* Quantise-and-append: the cache write that precedes the attention call (the
  * INT4 paged-KV page, Code analysis 2-3: per-channel symmetric codes,

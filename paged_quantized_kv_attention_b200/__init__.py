@@ -26,7 +26,7 @@ PA_NOALLOC_MAX_WORKSPACE_BYTES = 16 << 20
 EXPORTED = ["paged_attn_plan", "paged_attn_forward", "paged_attn_forward_noalloc",
             "paged_attn_workspace_init",
             "paged_attn_read_device_error", "paged_kv_pack_int4", "paged_kv_unpack_int4",
-            "paged_kv_gather_decode", "paged_kv_append", "paged_attn_stream_read",
+            "paged_kv_gather_decode", "paged_kv_append", "paged_attn_merge", "paged_attn_stream_read",
             "paged_attn_last_error", "paged_attn_version"]
 
 
@@ -49,7 +49,8 @@ class paged_attn_params(ctypes.Structure):  # noqa: N801 (mirrors the C struct n
                 ("num_row_groups", ctypes.c_int), ("num_splits", ctypes.c_int),
                 ("blocks_per_split", ctypes.c_int), ("num_work_items", ctypes.c_int),
                 ("workspace_bytes", ctypes.c_size_t),
-                ("workspace", ctypes.c_void_p), ("profile_events", ctypes.c_void_p)]
+                ("workspace", ctypes.c_void_p), ("profile_events", ctypes.c_void_p),
+                ("lse_out", ctypes.c_void_p)]
 
 
 _lib = None
@@ -74,6 +75,7 @@ def lib() -> ctypes.CDLL:
         L.paged_kv_unpack_int4.argtypes = [P, P, ctypes.c_int64, I, P]
         L.paged_kv_gather_decode.argtypes = [P, P, PP, I, I, I, I, P, P]
         L.paged_kv_append.argtypes = [P] * 9 + [PP, P]
+        L.paged_attn_merge.argtypes = [P, P, I, ctypes.c_int64, I, I, P, P, P]
         L.paged_attn_stream_read.argtypes = [P, S, P, P]
         L.paged_attn_last_error.restype = ctypes.c_char_p
         L.paged_attn_version.restype = ctypes.c_char_p
@@ -178,6 +180,13 @@ def paged_kv_append(k_new, v_new, k_cache, v_cache, k_scale, v_scale, block_tabl
     _check(lib().paged_kv_append(_ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
                                  _ptr(k_scale), _ptr(v_scale), _ptr(block_table), _ptr(seqlens_k),
                                  _ptr(cu_seqlens_q), ctypes.byref(params), _stream(stream)))
+
+
+def paged_attn_merge(parts, lse_parts, n_parts: int, rows: int, head_size: int, dtype: int, out,
+                     lse_out=None, stream=None):
+    """Log-sum-exp merge of results over disjoint key sets (see paged_attn.h)."""
+    _check(lib().paged_attn_merge(_ptr(parts), _ptr(lse_parts), n_parts, rows, head_size, dtype,
+                                  _ptr(out), _ptr(lse_out), _stream(stream)))
 
 
 def paged_attn_stream_read(src, nbytes: int, sink, stream=None):

@@ -352,6 +352,7 @@ pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_c
   a.o_part = p->num_splits > 1 ? reinterpret_cast<__half*>(ws + lay.o_part) : nullptr;
   a.lse_part = p->num_splits > 1 ? reinterpret_cast<float*>(ws + lay.lse_part) : nullptr;
   a.row_ns = p->num_splits > 1 ? reinterpret_cast<int32_t*>(ws + lay.row_ns) : nullptr;
+  a.lse_out = p->lse_out;
   a.batch = p->batch;
   a.H = p->num_heads;
   a.Hk = p->kv_num_heads;
@@ -508,6 +509,22 @@ pa_status paged_kv_append(const void* k_new, const void* v_new, void* k_cache, v
   a.in_bf16 = p->q_dtype == PA_BF16;
   cudaError_t e = pa::launch_append(p->kv_dtype, p->head_size, a, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ok() : cuda_status(e, "append launch");
+}
+
+pa_status paged_attn_merge(const void* parts, const float* lse_parts, int n_parts, int64_t rows,
+                           int head_size, int dtype, void* out, float* lse_out, void* stream) {
+  if (!parts || !lse_parts || !out) return fail(PA_ERR_INVALID_ARG, "NULL pointer argument");
+  if (n_parts < 1 || n_parts > 64) return fail(PA_ERR_INVALID_ARG, "n_parts %d not in [1, 64]", n_parts);
+  if (rows < 0) return fail(PA_ERR_INVALID_ARG, "rows < 0");
+  if (head_size != 64 && head_size != 128)
+    return fail(PA_ERR_UNSUPPORTED, "head_size %d not in {64, 128}", head_size);
+  if (dtype != PA_F16 && dtype != PA_BF16) return fail(PA_ERR_INVALID_ARG, "dtype must be PA_F16 or PA_BF16");
+  if (!aligned(parts, 8) || !aligned(out, 8) || !aligned(lse_parts, 4))
+    return fail(PA_ERR_INVALID_ARG, "parts/out must be 8-byte and lse_parts 4-byte aligned");
+  if (rows == 0) return ok();
+  cudaError_t e = pa::launch_merge(parts, lse_parts, n_parts, rows, head_size, dtype == PA_BF16, out,
+                                   lse_out, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ok() : cuda_status(e, "merge launch");
 }
 
 pa_status paged_attn_stream_read(const void* src, size_t bytes, void* sink, void* stream) {

@@ -179,4 +179,71 @@ cudaError_t launch_append(int kv_dtype, int head_size, const AppendArgs& a, cuda
   }
 }
 
+// ---------------------------------------------------------------------------
+// Log-sum-exp merge of results over disjoint key sets: one warp per row; lane p
+// holds part p's weight (n_parts <= 64: two per lane), then each lane sums its
+// dims over the parts.
+template <int D>
+__global__ void __launch_bounds__(128) pa_merge_kernel(const uint16_t* __restrict__ parts,
+                                                       const float* __restrict__ lse_parts,
+                                                       int n_parts, long long rows, bool bf16,
+                                                       uint16_t* __restrict__ out,
+                                                       float* __restrict__ lse_out) {
+  const int lane = threadIdx.x & 31;
+  const long long r = static_cast<long long>(blockIdx.x) * 4 + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  float l0 = lane < n_parts ? __ldg(lse_parts + static_cast<long long>(lane) * rows + r) : -INFINITY;
+  float l1 = lane + 32 < n_parts ? __ldg(lse_parts + static_cast<long long>(lane + 32) * rows + r)
+                                 : -INFINITY;
+  float M = fmaxf(l0, l1);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  const float w0 = (l0 == -INFINITY) ? 0.f : __expf(l0 - M);
+  const float w1 = (l1 == -INFINITY) ? 0.f : __expf(l1 - M);
+  float sum = w0 + w1;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const float inv = sum > 0.f ? 1.f / sum : 0.f;
+  if (lse_out != nullptr && lane == 0) lse_out[r] = sum > 0.f ? M + __logf(sum) : -INFINITY;
+  constexpr int kPairs = D / 2;  // half2 pairs per row
+  for (int d2 = lane; d2 < kPairs; d2 += 32) {
+    float ax = 0.f, ay = 0.f;
+    for (int pidx = 0; pidx < n_parts; ++pidx) {
+      const float wv = __shfl_sync(0xffffffffu, pidx < 32 ? w0 : w1, pidx & 31) * inv;
+      if (wv == 0.f) continue;  // empty part: its values are not read
+      const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(
+          parts + (static_cast<long long>(pidx) * rows + r) * D) + d2);
+      const float x = bf16 ? __uint_as_float(v << 16) : __half2float(__ushort_as_half(v & 0xFFFFu));
+      const float y = bf16 ? __uint_as_float(v & 0xFFFF0000u) : __half2float(__ushort_as_half(v >> 16));
+      ax = fmaf(wv, x, ax);
+      ay = fmaf(wv, y, ay);
+    }
+    uint32_t o;
+    if (bf16) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(ax, ay);
+      o = *reinterpret_cast<const uint32_t*>(&h);
+    } else {
+      const __half2 h = __floats2half2_rn(ax, ay);
+      o = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    reinterpret_cast<uint32_t*>(out + r * D)[d2] = o;
+  }
+}
+
+cudaError_t launch_merge(const void* parts, const float* lse_parts, int n_parts, long long rows,
+                         int head_size, bool bf16, void* out, float* lse_out, cudaStream_t stream) {
+  if (rows <= 0) return cudaSuccess;
+  const long long blocks = (rows + 3) / 4;
+  if (blocks >= (1ll << 31)) return cudaErrorInvalidValue;
+  const auto* pp = static_cast<const uint16_t*>(parts);
+  auto* op = static_cast<uint16_t*>(out);
+  if (head_size == 128)
+    pa_merge_kernel<128><<<static_cast<unsigned>(blocks), 128, 0, stream>>>(pp, lse_parts, n_parts,
+                                                                            rows, bf16, op, lse_out);
+  else
+    pa_merge_kernel<64><<<static_cast<unsigned>(blocks), 128, 0, stream>>>(pp, lse_parts, n_parts,
+                                                                           rows, bf16, op, lse_out);
+  return cudaGetLastError();
+}
+
 }  // namespace pa

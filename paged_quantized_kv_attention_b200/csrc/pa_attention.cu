@@ -1179,6 +1179,10 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
           }
           if (is_split && g == 0)
             a.lse_part[prow] = (L > 0.f) ? m_run[nt][j] + __log2f(L) : -INFINITY;
+          // the row's log-sum-exp for callers that merge results (natural log)
+          if (!is_split && a.lse_out != nullptr && g == 0)
+            a.lse_out[orow] = (L > 0.f) ? (m_run[nt][j] + __log2f(L)) * 0.6931471805599453f
+                                        : -INFINITY;
           // every row's split count, for the combine (1: stored above)
           if (a.row_ns != nullptr && split == 0 && g == 0) a.row_ns[orow] = nsplit;
         }
@@ -1262,6 +1266,8 @@ __global__ void __launch_bounds__(128) pa_combine_kernel(const FwdArgs a) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(kFull, sum, o);
   const float inv = sum > 0.f ? 1.f / sum : 0.f;
+  if (a.lse_out != nullptr && wsub == 0 && lane == 0)  // merged log-sum-exp (natural log)
+    a.lse_out[gr] = sum > 0.f ? (M + __log2f(sum)) * 0.6931471805599453f : -INFINITY;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int u0 = 0; wsub + WPR * u0 < S; u0 += kB) {
     if (u0 > 0) {  // splits beyond the first batch

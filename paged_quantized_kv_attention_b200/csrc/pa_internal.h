@@ -22,6 +22,7 @@ struct FwdArgs {
   __half* o_part;       // [max_splits, total_q * H, D] fp16, code units (split mode only)
   float* lse_part;      // [max_splits, total_q * H] (log2 domain)
   int32_t* row_ns;      // [total_q * H] splits with keys of each row's unit (split mode only)
+  float* lse_out;       // optional [total_q * H] natural-log log-sum-exp of each row
   uint32_t* frag;       // [batch * Hk * num_row_groups] precomputed query fragment units
   uint32_t* work;       // [2]: next work item, CTAs finished (both rewound by the last CTA)
   uint32_t* err;        // sticky device error word
@@ -76,6 +77,9 @@ struct AppendArgs {
   bool in_bf16;
 };
 cudaError_t launch_append(int kv_dtype, int head_size, const AppendArgs& a, cudaStream_t stream);
+// Log-sum-exp merge of results over disjoint key sets (pa_append.cu).
+cudaError_t launch_merge(const void* parts, const float* lse_parts, int n_parts, long long rows,
+                         int head_size, bool bf16, void* out, float* lse_out, cudaStream_t stream);
 
 // Launcher (pa_attention.cu).  rows_per_cta is 4 (decode rows packed with their
 // fp16 residuals), 8 or 16.

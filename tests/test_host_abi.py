@@ -226,6 +226,20 @@ def test_append_checks_arguments_before_any_launch():
     pa.paged_kv_append(*args, p0, stream=0)
 
 
+def test_merge_checks_arguments_before_any_launch():
+    buf = np.zeros(1024, dtype=np.uint8)
+    al = buf[(-buf.ctypes.data) % 16:]
+    for bad in (dict(n_parts=0), dict(n_parts=65), dict(head_size=96), dict(dtype=7)):
+        kw = dict(n_parts=2, head_size=128, dtype=pa.PA_F16)
+        kw.update(bad)
+        with pytest.raises(pa.PagedAttnError):
+            pa.paged_attn_merge(al, al, kw["n_parts"], 4, kw["head_size"], kw["dtype"], al, stream=0)
+    with pytest.raises(pa.PagedAttnError) as ei:
+        pa.paged_attn_merge(None, al, 2, 4, 128, pa.PA_F16, al, stream=0)
+    assert ei.value.status == pa.PA_ERR_INVALID_ARG
+    pa.paged_attn_merge(al, al, 2, 0, 128, pa.PA_F16, al, stream=0)  # no rows: nothing launched
+
+
 def test_codec_entry_points_check_arguments():
     with pytest.raises(pa.PagedAttnError):
         pa.paged_kv_pack_int4(None, None, 4, 128, stream=0)
