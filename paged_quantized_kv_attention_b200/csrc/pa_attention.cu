@@ -411,15 +411,20 @@ __global__ void __launch_bounds__(64) pa_prep_kernel(const FwdArgs a) {
   const int nrows = min(R, row0 + C::kRows) - row0;
   uint32_t qf[NT][C::kQWords];
   float crow[NT];
+  // the head's V scales must be finite too (checked once per sequence and head;
+  // loaded first so that their latency overlaps the fold)
+  float vsc[D / 32];
+#pragma unroll
+  for (int k = 0; k < D / 32; ++k)
+    vsc[k] = rg == 0 ? __ldg(a.v_scale + static_cast<size_t>(h) * D + 32 * k + lane) : 0.f;
   const uint8_t* qh = reinterpret_cast<const uint8_t*>(a.q) +
                       (static_cast<size_t>(q0) * a.H + static_cast<size_t>(h) * a.G) * D * 2;
   query_fragments<KV, D, BS, NT, LP>(a, qh, a.k_scale + static_cast<size_t>(h) * D, row0, nrows,
                                      lane, qf, crow);
-  if (rg == 0) {  // the head's V scales must be finite too (once per sequence and head)
-    bool ok = true;
-    for (int d = lane; d < D; d += 32) ok &= isfinite(__ldg(a.v_scale + static_cast<size_t>(h) * D + d));
-    if (__any_sync(kFull, !ok) && lane == 0) record_error(a.err, PA_DEVERR_BAD_SCALE);
-  }
+  bool v_ok = true;
+#pragma unroll
+  for (int k = 0; k < D / 32; ++k) v_ok &= isfinite(vsc[k]);
+  if (__any_sync(kFull, !v_ok) && lane == 0) record_error(a.err, PA_DEVERR_BAD_SCALE);
   uint32_t* fb = a.frag + static_cast<size_t>(u) * C::kUnitWords;
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
