@@ -47,7 +47,7 @@ EXTRA = ["c3_int8_long_split", "c5_fp8_large_batch", "c4_ragged_prefill_int8", "
 L2_FLUSH_BYTES = 256 << 20
 L2_BYTES = 126 << 20
 MAX_REPLICAS = 16
-SPIN_CYCLES = 200000  # ~0.1 ms of GPU work queued ahead of every timed span
+SPIN_CYCLES = 1000000  # ~0.5 ms of GPU work queued ahead of every timed span
 
 
 def algorithmic_bytes(w: dict) -> dict:
