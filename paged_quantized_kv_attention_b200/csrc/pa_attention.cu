@@ -1,5 +1,14 @@
 // pa_attention.cu -- fused paged quantised-KV GQA attention for sm_100a.
 //
+// A call is three kernels chained by programmatic dependent launch:
+//   pa_prep_kernel    folds each KV head's k_scale into its query rows and stores
+//                     every consumer lane's B-operand words (query digits or fp16
+//                     parts) and the rows' logit multipliers in the workspace,
+//                     once per (sequence, KV head, row group) unit;
+//   pa_fwd_kernel     the fused, persistent attention kernel (below);
+//   pa_combine_kernel the log-sum-exp merge of split partials (only when the
+//                     plan splits the KV).
+//
 // Work items.  An item is (sequence, group of 4 KV heads, group of query rows,
 // KV split).  The rows of one head are the (new token, query head of the GQA
 // group) pairs that read that head's keys; they form the N side of the
@@ -8,28 +17,30 @@
 // decoding), T chosen by the planner so that the items fill the resident CTAs.
 // Items are numbered densely over the sequences with new tokens: the producer
 // warp of every CTA computes the per-sequence item counts and their prefix sums
-// once, from the device lengths.  The kernel is persistent: CTA i starts with
-// item i and then pulls items from an atomic counter in the workspace.
+// once, from the device lengths, into a shared-memory table.  The kernel is
+// persistent: CTA i starts with item i and then pulls items from an atomic
+// counter in the workspace.
 //
 // Per CTA, one producer warp and four consumer warps, consumer warp w owning KV
 // head 4 hg + w of the item:
-//   producer : per item, bulk-copies the query rows and the k_scale rows of the
-//              four heads into the query buffer, then streams the item's KV in
-//              stages of 16 tokens: one 3-D TMA box (channels x 16 tokens x 4
-//              heads, heads outermost in shared memory) for K and one for V.
-//              Producer lane l owns ring stage l and refills it as soon as all
-//              four consumer warps have released it.
-//   consumers: per item, each warp folds its head's k_scale into its query rows
-//              and encodes them as B-operand fragments in registers, then for
-//              every stage: ldmatrix (its head's K rows) -> QK on the tensor cores
-//              -> online softmax (exp2 domain; the running maximum is raised only
+//   producer : per item, streams the KV in stages of 16 tokens: one 3-D TMA box
+//              (channels x 16 tokens x 4 heads, heads outermost in shared
+//              memory) for K and one for V into an mbarrier ring.  Producer lane
+//              l owns ring stage l and refills it as soon as all four consumer
+//              warps have released it; when no lane can issue, the warp sleeps
+//              on its oldest pending stage.
+//   consumers: per item, each warp loads its head's fragments (after the
+//              pre-pass grid completes, for the first item), then for every
+//              stage: ldmatrix (its head's K rows) -> QK on the tensor cores ->
+//              online softmax (exp2 domain; the running maximum is raised only
 //              when a logit exceeds it by more than 2^8) -> P^T in fp16 ->
-//              ldmatrix.trans (V) -> code -> fp16 -> PV MMA.  At the end the warp
-//              applies the V scale and stores its head's rows, or writes a split
-//              partial and its log2-sum-exp; the last split of a (sequence, head,
-//              row group) to finish merges the partials (arrival counter in the
-//              workspace).  No consumer barrier: the warps never wait on each
-//              other.
+//              ldmatrix.trans (V) -> code -> fp16 -> PV MMA.  With one n-tile the
+//              next stage's QK MMAs are issued before this stage's softmax and
+//              PV.  At the end the warp applies the V scale and stores its head's
+//              rows (and, on request, their log-sum-exps), or writes an fp16
+//              split partial in code units, its log2-sum-exp and the row's split
+//              count for the combine.  No consumer barrier: the warps never wait
+//              on each other.
 //
 // QK arithmetic.  INT8 and INT4 caches: the folded query q'' = q' 2^(6 - e_q)
 // (|q''| < 64) is split into signed int8 digits q'' = d0 + d1 2^-7 + d2 2^-14
