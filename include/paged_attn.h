@@ -28,6 +28,12 @@
  *  - "FlashInfer FP8 KV-Cache Prefill ... Repacking" (flashinfer PR 3485):
  *    1-byte FP8 KV cache (read here as OCP e4m3fn).
  *
+ * Besides the attention call the ABI has the cache writer that fills the cache
+ * (paged_kv_append: new fp16/bf16 K/V rows -> per-channel codes at their slots)
+ * and the log-sum-exp merge of results over disjoint key sets
+ * (paged_attn_merge, with the forward call's optional per-row lse_out) for a
+ * sequence whose keys are spread over several GPUs.
+ *
  * Readings where the pages are silent (all of them are properties of this ABI):
  *  - seqlens_k[b] counts every key of sequence b, the new tokens included; the
  *    past length is seqlens_k[b] - q_b (q_b = new tokens of b).
@@ -63,8 +69,8 @@
  * any launch and return PA_ERR_INVALID_ARG / PA_ERR_UNSUPPORTED /
  * PA_ERR_WORKSPACE.  A launch failure returns PA_ERR_CUDA.  Conditions that
  * only the device can see (a block-table entry outside [0, num_blocks), a
- * non-finite k_scale, device lengths that contradict the plan, a pipeline wait
- * that timed out) never fault the GPU: the kernel reads zeros instead, finishes,
+ * non-finite K or V scale, device lengths that contradict the plan, a pipeline
+ * wait that timed out) never fault the GPU: the kernel reads zeros instead, finishes,
  * and ORs a bit into the sticky error word at the start of the workspace, which
  * paged_attn_read_device_error() returns.
  */
