@@ -115,6 +115,24 @@ def test_edge_lengths(kv, lens):
             _check(w, out)
 
 
+@pytest.mark.parametrize("kv", ALL_KV)
+@pytest.mark.parametrize("B,qmax,D", [(300, 1, 64), (170, 4, 128)])
+def test_many_sequences_use_the_sparse_item_numbering(kv, B, qmax, D):
+    """More sequences than the producer's shared-memory item table holds (256, or
+    160 for the two-n-tile kernels with 128-byte rows): every sequence gets the
+    largest item count and empty items are skipped.  Zero-new-token sequences mixed
+    in; decode (300 sequences) and up to 16 rows per KV head (170 sequences)."""
+    rng = np.random.default_rng(B + kv)
+    ql = rng.integers(0, qmax + 1, size=B)
+    lens = rng.integers(1, 60, size=B) + ql
+    prob, _ = paged_problem(rng, kv_dtype=kv, lens=lens.tolist(), q_lens=ql.tolist(), H=8, Hk=2,
+                            D=D, bs=16)
+    w = _as_workload(prob, q_dtype=0, out_dtype=0)
+    out, p, ws = _gpu.run(w)
+    assert pa.paged_attn_read_device_error(ws)[1] == 0
+    _check(w, out)
+
+
 def _as_workload(prob, q_dtype, out_dtype):
     w = dict(prob)
     w["q"] = torch.from_numpy(prob["q"]).to(torch.bfloat16 if q_dtype else torch.float16)
