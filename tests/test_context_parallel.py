@@ -37,6 +37,31 @@ def test_shard_ranges_partition_every_sequence():
             assert max(sizes) - min(sizes) <= 1
 
 
+@pytest.mark.parametrize("world", [2, 3, 5])
+def test_local_problems_rebuild_the_full_attention(world):
+    """Host-side rank views: each rank's block table, lengths and rows, run through
+    the oracle as an ordinary problem, merge (oracle combine) into the unsplit
+    attention (1e-12); a rank without keys for a sequence gets no rows for it."""
+    prob = _problem(31, lens=(300, 47, 1000, 17, 5))
+    T, H, D = int(prob["cu_seqlens_q"][-1]), prob["num_heads"], prob["head_size"]
+    ranges = cp.shard_ranges(prob["seqlens_k"], prob["block_size"], world)
+    parts = np.zeros((world, T, H, D))
+    lses = np.full((world, T, H), -np.inf)
+    for r in range(world):
+        lbt, lL, lcu, rows = cp.local_problem(prob["block_table"], prob["cu_seqlens_q"], ranges[r],
+                                              prob["block_size"])
+        assert len(rows) == int(lcu[-1])
+        if len(rows) == 0:
+            continue
+        loc = dict(prob, block_table=lbt, seqlens_k=lL, cu_seqlens_q=lcu,
+                   max_blocks_per_seq=lbt.shape[1], q=prob["q"][rows])
+        o, l = oracle.paged_attn_partial(loc, np.zeros_like(lL), lL)
+        parts[r, rows], lses[r, rows] = o, l
+    merged = oracle.lse_combine(parts.reshape(world, T * H, D), lses.reshape(world, T * H))
+    ref = oracle.paged_attn(prob)
+    assert np.max(np.abs(merged.reshape(T, H, D) - ref)) <= 1e-12 * np.max(np.abs(ref))
+
+
 def _oracle_rank(prob, ranges_r):
     """Rank-local (output, lse) rows from the oracle's partial attention."""
     o, lse = oracle.paged_attn_partial(prob, ranges_r[:, 0], ranges_r[:, 1])
