@@ -6,15 +6,19 @@
 //
 // The code of a value is decided in IEEE single precision: q = x * inv, inv the
 // fp32-rounded inverse of the channel's scale, then INT8: nearest integer, ties
-// to even, clamped to
-// [-127, 127]; INT4: the same clamped to [-8, 7], channel 2j in the low nibble of
-// byte j; FP8: round-to-nearest-even e4m3fn, saturating at +-448.  A NaN quotient
-// stores 0 (integer caches) or 0x7F (FP8).
+// to even, clamped to [-127, 127]; INT4: the same clamped to [-8, 7], channel 2j
+// in the low nibble of byte j; FP8: round-to-nearest-even e4m3fn, saturating at
+// +-448.  A NaN quotient stores 0 (integer caches) or 0x7F (FP8).
 //
-// HBM-bound and elementwise: a warp takes one new token's K or V rows; lane l
+// HBM-bound and elementwise: a warp takes one new token's K and V rows; lane l
 // handles 8-channel groups l, l + 32, ... of the token's Hk x D values (16 bytes
 // of fp16/bf16 in, 8 or 4 bytes out), so both the reads and the row writes of a
-// token (its heads are contiguous in the cache slot) are contiguous.
+// token (its heads are contiguous in the cache slot) are contiguous.  The
+// per-channel inverse scales sit in shared memory.
+//
+// Also here: the log-sum-exp merge of attention results over disjoint key sets
+// (context parallelism; the flash-decoding combine of the GQA GEMV decode page,
+// onnxruntime PR 29216, Code analysis 2).
 #include <cuda_fp8.h>
 
 #include "pa_device.cuh"
