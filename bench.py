@@ -11,9 +11,13 @@ every step reads its KV cache from HBM; a workload too small for that (the tiny
 case) instead flushes L2 by writing a 256 MB buffer before each step, outside the
 timed span.  Each step is timed with CUDA events on the launching stream.
 
-Headline workload (N=1): INT4 packed decode, B=16, q_len=1, 32 query / 8 KV
-heads, head_size 128, block_size 16, seqlens_k ~ U[512, 4096].  The other
-workloads are reported under "workloads" with the same method.
+Headline workload (N=1): the largest configuration, FP8 e4m3 large-batch decode,
+B=128, q_len=1, 64 query / 8 KV heads, head_size 128, block_size 16, seqlens_k =
+8192 (2.15 GB of KV per call).  The other workloads (INT4 decode, INT8 long-context
+split decode, INT8 ragged causal prefill, the tiny INT8 case, the cache writer)
+are reported under "workloads" with the same method, each with its own roofline
+block.  A read-only 16-byte-vector stream over a 2 GiB buffer
+(paged_attn_stream_read) is timed beside them as the measured read ceiling.
 
 Metric: effective HBM bandwidth = algorithmic bytes per call / time per call
 (KV bytes of the sequences with new tokens + Q in + out + scales + block-table
@@ -42,8 +46,8 @@ import torch  # noqa: E402
 
 import workloads  # noqa: E402
 
-HEADLINE = "c2_int4_decode"
-EXTRA = ["c3_int8_long_split", "c5_fp8_large_batch", "c4_ragged_prefill_int8", "c1_tiny_int8"]
+HEADLINE = "c5_fp8_large_batch"
+EXTRA = ["c2_int4_decode", "c3_int8_long_split", "c4_ragged_prefill_int8", "c1_tiny_int8"]
 L2_FLUSH_BYTES = 256 << 20
 L2_BYTES = 126 << 20
 MAX_REPLICAS = 16
@@ -99,6 +103,88 @@ def measured_peaks():
         return float(pk["hbm_gbs"]), "measured"
     except (OSError, ValueError, KeyError):
         return 6650.0, "fallback"
+
+
+def measured_tensor_peak():
+    """Dense bf16 tensor peak (TFLOP/s, burst) of MEASURED_PEAKS.json, else the
+    fallback figure."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except (OSError, ValueError, KeyError):
+        return 1590.0, "fallback"
+
+
+def algorithmic_flops(w: dict) -> int:
+    """Useful tensor work per call: 2 D flops for QK and 2 D for PV per visible
+    key of every row (rows = new tokens x query heads; causal rows see their
+    past plus the new tokens up to themselves)."""
+    D, H = w["head_size"], w["num_heads"]
+    cu = w["cu_seqlens_q"].astype(np.int64)
+    L = w["seqlens_k"].astype(np.int64)
+    keys = 0
+    for b in range(w["batch"]):
+        qb = int(cu[b + 1] - cu[b])
+        if qb == 0:
+            continue
+        past = int(L[b]) - qb
+        if w["causal"]:
+            keys += qb * past + qb * (qb + 1) // 2
+        else:
+            keys += qb * int(L[b])
+    return 4 * D * H * keys
+
+
+def roofline_block(w: dict, ab: dict, kern_ms: float, name: str) -> dict:
+    """Roofline of the call's kernels for one workload: bound = the larger of the
+    HBM time (algorithmic bytes / measured copy peak) and the tensor time
+    (algorithmic flops / measured bf16 peak); achieved in that bound's unit."""
+    peak, kind = measured_peaks()
+    tpk, tkind = measured_tensor_peak()
+    flops = algorithmic_flops(w)
+    t_hbm = ab["total"] / (peak * 1e9)
+    t_mma = flops / (tpk * 1e12)
+    sec = kern_ms * 1e-3
+    if t_mma > t_hbm:
+        return {"bound": "tensor", "achieved": round(flops / sec / 1e12, 2), "peak": tpk,
+                "unit": "TFLOP/s", "frac": round(t_mma / sec, 4), "peak_kind": tkind,
+                "algorithmic_flops_per_launch": flops, "traffic": ncu_traffic(name)}
+    return {"bound": "hbm", "achieved": round(ab["total"] / sec / 1e9, 1), "peak": peak,
+            "unit": "GB/s", "frac": round(t_hbm / sec, 4), "peak_kind": kind,
+            "algorithmic_bytes_per_launch": ab["total"], "algorithmic_flops_per_launch": flops,
+            "frac_of_tensor_peak": round(t_mma / sec, 4), "traffic": ncu_traffic(name)}
+
+
+READ_CEILING_BYTES = 2 << 30
+
+
+def read_ceiling(dev: str, steps: int = 10) -> dict:
+    """Measured read-only ceiling: paged_attn_stream_read (16-byte loads on every
+    SM) over a 2 GiB buffer, CUDA events on the launching stream, best and mean
+    of `steps` launches after 3 warm-up launches."""
+    import paged_quantized_kv_attention_b200 as pa
+    buf = torch.empty(READ_CEILING_BYTES, dtype=torch.uint8, device=dev)
+    buf.fill_(1)
+    sink = torch.empty(16 * 148 * 64, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(3):
+        pa.paged_attn_stream_read(buf, READ_CEILING_BYTES, sink, stream)
+    ms = []
+    for _ in range(steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        pa.paged_attn_stream_read(buf, READ_CEILING_BYTES, sink, stream)
+        e1.record(stream)
+        e1.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    del buf
+    torch.cuda.empty_cache()
+    peak, kind = measured_peaks()
+    best = READ_CEILING_BYTES / (min(ms) * 1e-3) / 1e9
+    mean = READ_CEILING_BYTES / (statistics.mean(ms) * 1e-3) / 1e9
+    return {"kernel": "pa_stream_read_kernel (paged_attn_stream_read)", "bytes": READ_CEILING_BYTES,
+            "gbs_best": round(best, 1), "gbs_mean": round(mean, 1),
+            "vs_%s_copy_peak" % kind: round(mean / peak, 4)}
 
 
 class ClockSampler:
@@ -336,8 +422,24 @@ def sub_problem(w: dict, b: int) -> dict:
     return s
 
 
-def measure(name: str, steps: int, warmup: int, dev: str, flush_buf, with_e2e: bool):
-    w = workloads.make(name)
+def first_sequences(w: dict, B: int) -> dict:
+    """The workload cut to its first B sequences (same cache pools, heads and
+    dtypes): a smaller instance of the same shape, for profiler captures."""
+    if B is None or B >= w["batch"]:
+        return w
+    s = dict(w)
+    cu = w["cu_seqlens_q"]
+    s["batch"] = B
+    s["block_table"] = np.ascontiguousarray(w["block_table"][:B])
+    s["seqlens_k"] = np.ascontiguousarray(w["seqlens_k"][:B])
+    s["cu_seqlens_q"] = np.ascontiguousarray(cu[:B + 1])
+    s["q"] = w["q"][:int(cu[B])]
+    return s
+
+
+def measure(name: str, steps: int, warmup: int, dev: str, flush_buf, with_e2e: bool,
+            batch=None):
+    w = first_sequences(workloads.make(name), batch)
     ab = algorithmic_bytes(w)
     replicas, use_flush = l2_plan(w)
     flush = flush_buf if use_flush else None
@@ -430,7 +532,9 @@ def summary_of(name, r):
             "kernel_us": round(r["kern_ms"] * 1e3, 2),
             "kernel_gbs": round(r["kernel_gbs"], 1),
             "kernel_frac_of_%s_peak" % r["peak_kind"]: round(r["kernel_gbs"] / r["peak"], 3),
-            "num_splits": r["p"].num_splits, "algorithmic_bytes": r["ab"]["total"], "l2": r["l2"]}
+            "num_splits": r["p"].num_splits, "algorithmic_bytes": r["ab"]["total"], "l2": r["l2"],
+            "launches_per_call": r["launches_per_step"],
+            "roofline": roofline_block(r["w"], r["ab"], r["kern_ms"], name)}
 
 
 def run_ours(args):
@@ -458,7 +562,7 @@ def run_ours(args):
         dist.barrier()
     torch.cuda.synchronize()
     with sampler:
-        r = measure(w_name, args.steps, args.warmup, dev, flush, with_e2e=True)
+        r = measure(w_name, args.steps, args.warmup, dev, flush, with_e2e=True, batch=args.batch)
     torch.cuda.synchronize()
     if dist is not None:
         t = torch.tensor([r["call_ms"], r["e2e"]["ms_per_step"]], device=dev)
@@ -466,7 +570,9 @@ def run_ours(args):
         dist.barrier()
         r["call_ms"], r["e2e"]["ms_per_step"] = float(t[0]), float(t[1])
     extra = {}
+    ceiling = None
     if not args.no_extra:
+        ceiling = read_ceiling(dev)
         for name in EXTRA:
             if name == w_name:
                 continue
@@ -485,17 +591,21 @@ def run_ours(args):
     cpu = None
     if world == 1 and not args.no_cpu:
         gbs, det = cpu_oracle_sample(r["w"], args.cpu_seconds)
-        cpu = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
-               "sample": "FP64 oracle, one thread, whole sequences of the same workload in order "
-                         "until ~%.0f s: %d sequences, %d keys, %.1f s" %
-                         (args.cpu_seconds, det["sequences"], det["keys"], det["seconds"])}
+        cpu = {"value": gbs, "unit": "GB/s", "cores": 1, "host_cores": os.cpu_count(),
+               "kind": "oracle",
+               "sample": "FP64 oracle, one thread (of %d host cores), whole sequences of the "
+                         "same workload in order until ~%.0f s: %d sequences, %d keys, %.1f s" %
+                         (os.cpu_count(), args.cpu_seconds, det["sequences"], det["keys"],
+                          det["seconds"])}
     line = {
         "metric": "paged quantized-KV attention: effective HBM GB/s (% of ~8 TB/s), us/call",
         "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(r["call_ms"], 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f16",
         "data": "synthetic (seeded numpy PCG64; cache resident in HBM)",
-        "config": {"workload": w_name, "desc": workloads.DESCRIPTIONS[w_name],
+        "config": {"workload": w_name if args.batch is None else
+                   "%s (first %d sequences)" % (w_name, r["w"]["batch"]),
+                   "desc": workloads.DESCRIPTIONS[w_name],
                    "kv_dtype": workloads.KV_NAMES[r["w"]["kv_dtype"]],
                    "global_batch": r["w"]["batch"] * world, "seq_len": int(r["w"]["seqlens_k"].max()),
                    "parallelism": "replicas x%d" % world,
@@ -509,15 +619,12 @@ def run_ours(args):
                 "d2h_bytes_per_step": r["e2e"]["d2h_bytes_per_step"],
                 "us_per_step": round(r["e2e"]["ms_per_step"] * 1e3, 2)},
         "gpu_launches": args.steps * r["launches_per_step"],
-        "roofline": {"bound": "hbm", "achieved": round(r["kernel_gbs"], 1),
-                     "peak": r["peak"], "unit": "GB/s",
-                     "frac": round(r["kernel_gbs"] / r["peak"], 4),
-                     "peak_kind": r["peak_kind"],
-                     "kernel": "pa_fwd_kernel (timed with its fragment pre-pass and, when "
-                               "split, its combine: the whole call on the device)",
-                     "kernel_us": round(r["kern_ms"] * 1e3, 3),
-                     "algorithmic_bytes_per_launch": ab["fwd"],
-                     "traffic": ncu_traffic(w_name)},
+        "roofline": dict(roofline_block(r["w"], ab, r["kern_ms"], w_name),
+                         kernel="pa_fwd_kernel (timed with the other kernels of the call, "
+                                "which overlap it: the whole call on the device)",
+                         kernel_us=round(r["kern_ms"] * 1e3, 3),
+                         read_ceiling_gbs=ceiling["gbs_mean"] if ceiling else None),
+        "read_ceiling": ceiling,
         "clocks": sampler.summary(),
         "cpu_baseline": cpu,
         "workloads": extra,
@@ -575,6 +682,9 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--batch", type=int, default=None,
+                    help="cut the workload to its first BATCH sequences (a smaller instance "
+                         "of the same shape, for profiler captures; not a bench line)")
     ap.add_argument("--writer", action="store_true",
                     help="time only the quantise-and-append writer workloads (one JSON line)")
     args = ap.parse_args()

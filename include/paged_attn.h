@@ -206,12 +206,16 @@ pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_c
  *    PA_NOALLOC_MAX_WORKSPACE_BYTES the call returns PA_ERR_WORKSPACE before any
  *    device work (plan again with a larger split_blocks, i.e. fewer splits, or
  *    use paged_attn_forward with your own workspace).
- *  - The first call on a device looks up the array's device address on that
- *    device (cudaGetSymbolAddress, the device current); make that first call
- *    before any stream capture on the device.
+ *  - Every call looks up the array's device address on the current device
+ *    (cudaGetSymbolAddress, a host-side query that allocates nothing).  The
+ *    first lookup on a device loads the library's device code there: make the
+ *    first call on a device before any stream capture on it.
  *  - Every call clears the array's error word and counters on `stream`
  *    (cudaMemsetAsync) before the launch; the array keeps the rest of the last
- *    call's contents.  There is no device-error readback for this path.
+ *    call's contents.  paged_attn_read_device_error(NULL, ...) reads (and
+ *    optionally clears) the array's error word on the current device, so the
+ *    device-side conditions of the last call are visible until the next call
+ *    clears them.
  *  - All calls in the process share the one array per device: calls whose
  *    executions overlap on the GPU (different streams without ordering between
  *    them) race on it and give wrong results.  Order them on one stream. */
@@ -226,9 +230,13 @@ pa_status paged_attn_forward_noalloc(const void* q, const void* k_cache, const v
 pa_status paged_attn_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronise `stream`, read the device error word from `workspace` into *bits
- * (PA_DEVERR_* flags), and zero it when `clear` is non-zero.  Returns PA_OK when
- * no bit is set, PA_ERR_BAD_BLOCK_TABLE when PA_DEVERR_BAD_BLOCK is set, and
- * PA_ERR_DEVICE for any other bit. */
+ * (PA_DEVERR_* flags), and zero it when `clear` is non-zero.  workspace NULL
+ * reads the word of paged_attn_forward_noalloc's library-owned scratch on the
+ * current device.  Returns PA_OK when no bit is set, PA_ERR_BAD_BLOCK_TABLE
+ * when PA_DEVERR_BAD_BLOCK is set, and PA_ERR_DEVICE for any other bit.  After
+ * PA_DEVERR_BAD_LENGTH (device lengths that contradict the plan) the rows of the
+ * offending sequences are undefined: out may hold values left from an earlier
+ * call sharing the workspace. */
 pa_status paged_attn_read_device_error(void* workspace, int clear, uint32_t* bits, void* stream);
 
 /* INT4 codec (INT4 paged-KV page, Code analysis 2).  pack: int8 values in

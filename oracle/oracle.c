@@ -361,10 +361,10 @@ static int encode_e4m3(float q) {
 }
 
 int oracle_quantise(int kv_dtype, float x, float s) {
-  /* IEEE single precision, no contraction: the inverse scale rounded to fp32,
-   * then the rounded product */
-  const float inv = 1.0f / s;
-  const float q = x * inv;
+  /* The symmetric code of x is the nearest code to x / s (value = scale x code),
+   * with the quotient taken in IEEE single precision: one correctly rounded
+   * division, no contraction. */
+  const float q = x / s;
   if (kv_dtype == ORACLE_KV_FP8_E4M3) return encode_e4m3(q);
   if (isnan(q)) return 0;
   const int lo = kv_dtype == ORACLE_KV_INT4 ? -8 : -127;

@@ -123,20 +123,20 @@ int oracle_lse_combine(int n_splits, int64_t rows, int head_size, const double* 
 /* Cache code of one new value x under per-channel scale s, for the
  * quantise-and-append writer that fills the cache the attention reads (INT4
  * paged-KV page, Code analysis 2: the cache holds per-channel symmetric codes,
- * value = scale x code).  The code is decided in IEEE single precision, the
- * writer's own arithmetic: q = (float)x * inv with inv = 1 / s rounded to fp32
- * (a multiply by the per-channel inverse scale), then
+ * value = scale x code).  The code is the nearest code to the quotient x / s,
+ * the plain definition of a symmetric code, with the quotient taken in IEEE
+ * single precision (one correctly rounded division):
  *   INT8: nearest integer to q (ties to even), clamped to [-127, 127];
  *   INT4: the same, clamped to [-8, 7] (the two's complement nibble);
  *   FP8 : the OCP e4m3fn value nearest to q (ties to the even mantissa),
  *         magnitudes past 448 saturated to 448; the sign of q is kept on 0.
  * A NaN quotient gives code 0 (integer caches) or 0x7F (FP8).  Readings (the
  * pages give the format, not the rounding): round to nearest even, symmetric
- * INT8 range, saturation, the inverse-scale multiply (one rounding of 1/s,
- * one of the product; a correctly rounded x / s would differ from it only at
- * rare rounding boundaries).  Returns the signed code (INT8 / INT4) or the byte
- * (FP8).  Pinned by: exact codes at power-of-two scales, ties, saturation,
- * the decode table round trip, torch's e4m3fn cast. */
+ * INT8 range, saturation, the quotient rounded once to fp32.  Returns the
+ * signed code (INT8 / INT4) or the byte (FP8).  Pinned by: exact codes at
+ * power-of-two scales, ties, saturation, the decode table round trip, torch's
+ * e4m3fn cast, and codes next to a rounding boundary decided from the exact
+ * rational quotient (where x times a rounded 1 / s lands on the other side). */
 int oracle_quantise(int kv_dtype, float x, float s);
 
 /* Quantise-and-append: the new K and V rows of every sequence ([T_q, Hk, D]

@@ -150,7 +150,8 @@ def paged_attn_workspace_init(workspace, nbytes: int, stream=None):
 
 
 def paged_attn_read_device_error(workspace, clear: bool = True, stream=None):
-    """(status, bits) of the sticky device error word; never raises for set bits."""
+    """(status, bits) of the sticky device error word; never raises for set bits.
+    ``workspace`` None reads the word of paged_attn_forward_noalloc's scratch."""
     bits = ctypes.c_uint32(0)
     st = lib().paged_attn_read_device_error(_ptr(workspace), int(clear), ctypes.byref(bits),
                                             _stream(stream))

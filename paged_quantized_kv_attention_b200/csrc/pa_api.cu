@@ -400,8 +400,12 @@ pa_status paged_attn_workspace_init(void* workspace, size_t workspace_bytes, voi
 }
 
 pa_status paged_attn_read_device_error(void* workspace, int clear, uint32_t* bits, void* stream) {
-  if (workspace == nullptr || bits == nullptr)
-    return fail(PA_ERR_INVALID_ARG, "workspace or bits is NULL");
+  if (bits == nullptr) return fail(PA_ERR_INVALID_ARG, "bits is NULL");
+  if (workspace == nullptr) {
+    // the error word of paged_attn_forward_noalloc's scratch on this device
+    const pa_status st = pa::noalloc_scratch_address(&workspace);
+    if (st != PA_OK) return st;
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint32_t word = 0;
   cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, s);
@@ -488,7 +492,7 @@ pa_status paged_kv_append(const void* k_new, const void* v_new, void* k_cache, v
     return fail(PA_ERR_WORKSPACE, "a 256-byte aligned workspace of >= 256 bytes holds the error word");
   if (static_cast<int64_t>(p->kv_num_heads) * p->head_size * 8 > 200 * 1024)
     return fail(PA_ERR_UNSUPPORTED, "kv_num_heads x head_size too large for the writer's "
-                "shared-memory inverse scales");
+                "shared-memory scales");
   pa::AppendArgs a;
   a.k_new = k_new;
   a.v_new = v_new;

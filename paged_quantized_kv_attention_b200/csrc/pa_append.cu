@@ -4,17 +4,18 @@
 // format of the INT4 paged-KV page, onnxruntime PR 32515, Code analysis 2-3)
 // and stored at the slot the block table gives their absolute position.
 //
-// The code of a value is decided in IEEE single precision: q = x * inv, inv the
-// fp32-rounded inverse of the channel's scale, then INT8: nearest integer, ties
-// to even, clamped to [-127, 127]; INT4: the same clamped to [-8, 7], channel 2j
-// in the low nibble of byte j; FP8: round-to-nearest-even e4m3fn, saturating at
-// +-448.  A NaN quotient stores 0 (integer caches) or 0x7F (FP8).
+// The code of a value is the code nearest to x / s, the quotient taken in IEEE
+// single precision (one correctly rounded division), then INT8: nearest
+// integer, ties to even, clamped to [-127, 127]; INT4: the same clamped to
+// [-8, 7], channel 2j in the low nibble of byte j; FP8: round-to-nearest-even
+// e4m3fn, saturating at +-448.  A NaN quotient stores 0 (integer caches) or
+// 0x7F (FP8).
 //
 // HBM-bound and elementwise: a warp takes one new token's K and V rows; lane l
 // handles 8-channel groups l, l + 32, ... of the token's Hk x D values (16 bytes
 // of fp16/bf16 in, 8 or 4 bytes out), so both the reads and the row writes of a
 // token (its heads are contiguous in the cache slot) are contiguous.  The
-// per-channel inverse scales sit in shared memory.
+// per-channel scales sit in shared memory.
 //
 // Also here: the log-sum-exp merge of attention results over disjoint key sets
 // (context parallelism; the flash-decoding combine of the GQA GEMV decode page,
@@ -31,10 +32,11 @@ __device__ __forceinline__ float bits_to_float(uint32_t h, bool bf16) {
               : __half2float(__ushort_as_half(static_cast<unsigned short>(h)));
 }
 
-// x times the inverse scale inv = 1 / s (rounded to fp32 once per channel).
+// Code of x under scale s: the correctly rounded fp32 quotient x / s, rounded
+// to the cache format.
 template <int KV>
-__device__ __forceinline__ uint32_t code_of(float x, float inv) {
-  const float q = __fmul_rn(x, inv);
+__device__ __forceinline__ uint32_t code_of(float x, float s) {
+  const float q = __fdiv_rn(x, s);
   if constexpr (KV == PA_KV_FP8_E4M3) {
     if (q != q) return 0x7Fu;
     return static_cast<uint32_t>(__nv_cvt_float_to_fp8(q, __NV_SATFINITE, __NV_E4M3)) & 0xFFu;
@@ -51,7 +53,7 @@ __device__ __forceinline__ uint32_t code_of(float x, float inv) {
 // or 8 bytes (INT8, FP8) in the low bits of out.
 template <int KV>
 __device__ __forceinline__ uint2 codes8(uint4 raw, float4 s0, float4 s1, bool bf16) {
-  const float s[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};  // inverse scales
+  const float s[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};  // channel scales
   const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
   uint32_t c[8];
 #pragma unroll
@@ -78,12 +80,12 @@ __global__ void __launch_bounds__(256) pa_append_kernel(AppendArgs a) {
   constexpr int kGroups = D / 8;
   constexpr int kChs = KV == PA_KV_INT4 ? D / 2 : D;
   constexpr int kU = 4;  // groups per lane per pass (of K and of V)
-  // inverse scales of every channel, K then V: [2][Hk][D] fp32
-  extern __shared__ float4 inv_s[];
-  float* inv = reinterpret_cast<float*>(inv_s);
+  // scales of every channel, K then V: [2][Hk][D] fp32
+  extern __shared__ float4 sc_s[];
+  float* sc = reinterpret_cast<float*>(sc_s);
   for (int i = threadIdx.x; i < a.Hk * D; i += blockDim.x) {
-    inv[i] = __frcp_rn(__ldg(a.k_scale + i));
-    inv[a.Hk * D + i] = __frcp_rn(__ldg(a.v_scale + i));
+    sc[i] = __ldg(a.k_scale + i);
+    sc[a.Hk * D + i] = __ldg(a.v_scale + i);
   }
   __syncthreads();
   const int lane = threadIdx.x & 31;
@@ -131,8 +133,8 @@ __global__ void __launch_bounds__(256) pa_append_kernel(AppendArgs a) {
         const int gi = g0 + 32 * u + lane;
         if (gi >= per_tok) break;
         // channels gi * 8 .. gi * 8 + 7 of the token's Hk x D row set
-        const float4* ki = inv_s + 2 * gi;
-        const float4* vi = inv_s + (a.Hk * D) / 4 + 2 * gi;
+        const float4* ki = sc_s + 2 * gi;
+        const float4* vi = sc_s + (a.Hk * D) / 4 + 2 * gi;
         const uint2 kc = codes8<KV>(kr[u], ki[0], ki[1], a.in_bf16);
         const uint2 vc = codes8<KV>(vr[u], vi[0], vi[1], a.in_bf16);
         // group gi is bytes [gi * 8, gi * 8 + 8) of the slot's Hk rows (INT4: 4)

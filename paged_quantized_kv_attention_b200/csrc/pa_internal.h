@@ -96,6 +96,10 @@ int fragment_unit_words(int kv_dtype, int head_size, int rows_per_cta);
 // Forward CTAs resident per SM, from the launch bounds and shared memory.
 int forward_ctas_per_sm(int kv_dtype, int head_size, int block_size, int rows_per_cta);
 
+// Device address, on the current device, of the library-owned scratch that
+// paged_attn_forward_noalloc uses as its workspace (pa_noalloc.cu).
+pa_status noalloc_scratch_address(void** out);
+
 // Sets the thread's message for paged_attn_last_error() and returns st
 // (pa_api.cu; used by entry points defined in other files).
 pa_status set_last_error(pa_status st, const char* msg);

@@ -17,8 +17,6 @@
 #include <stdarg.h>
 #include <stdio.h>
 
-#include <mutex>
-
 #include "pa_internal.h"
 
 namespace {
@@ -26,10 +24,6 @@ namespace {
 // The shared scratch.  In host code this name is only a host-side handle of the
 // symbol, not a device address; the address comes from cudaGetSymbolAddress.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[PA_NOALLOC_MAX_WORKSPACE_BYTES];
-
-constexpr int kMaxDevices = 64;
-std::mutex g_addr_mutex;
-void* g_addr[kMaxDevices] = {};
 
 // Records the message that paged_attn_last_error() returns on this thread.
 pa_status noalloc_fail(pa_status st, const char* fmt, ...) {
@@ -41,29 +35,25 @@ pa_status noalloc_fail(pa_status st, const char* fmt, ...) {
   return pa::set_last_error(st, msg);
 }
 
-// Device address of the scratch on the current device, looked up once per
-// device (with that device current) and cached.
-pa_status scratch_address(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess)
-    return noalloc_fail(PA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
-  if (dev < 0 || dev >= kMaxDevices)
-    return noalloc_fail(PA_ERR_UNSUPPORTED, "device ordinal %d >= %d", dev, kMaxDevices);
-  std::lock_guard<std::mutex> lock(g_addr_mutex);
-  if (g_addr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || p == nullptr)
-      return noalloc_fail(PA_ERR_CUDA, "cudaGetSymbolAddress(scratch) on device %d: %s", dev,
-                          cudaGetErrorString(e));
-    g_addr[dev] = p;
+}  // namespace
+
+// Device address of the scratch on the current device.  Looked up on every call
+// (a host-side query that allocates nothing): a cached address would dangle
+// after the device's context is torn down and created again.  The first lookup
+// on a device loads the library's device code there, which is why the first
+// call should come before any stream capture.
+pa_status pa::noalloc_scratch_address(void** out) {
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess || p == nullptr) {
+    int dev = -1;
+    cudaGetDevice(&dev);
+    return noalloc_fail(PA_ERR_CUDA, "cudaGetSymbolAddress(scratch) on device %d: %s", dev,
+                        cudaGetErrorString(e));
   }
-  *out = g_addr[dev];
+  *out = p;
   return PA_OK;
 }
-
-}  // namespace
 
 extern "C" {
 
@@ -86,7 +76,7 @@ pa_status paged_attn_forward_noalloc(const void* q, const void* k_cache, const v
     return paged_attn_forward(q, k_cache, v_cache, k_scale, v_scale, block_table, seqlens_k,
                               cu_seqlens_q, out, params, stream);  // no launch, no scratch
   void* scratch = nullptr;
-  pa_status st = scratch_address(&scratch);
+  pa_status st = pa::noalloc_scratch_address(&scratch);
   if (st != PA_OK) return st;
 
   // The array keeps the previous call's contents.  Zero what the kernel expects

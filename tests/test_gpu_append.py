@@ -94,6 +94,42 @@ def test_append_ties_and_specials(kv):
     np.testing.assert_array_equal(vc, vo)
 
 
+@pytest.mark.parametrize("kv", ALL_KV)
+def test_append_codes_next_to_a_rounding_boundary(kv):
+    """Inputs whose exact quotient x / s sits just past a boundary between two
+    codes, where x times a rounded 1 / s would store the neighbouring code: the
+    kernel stores the code of the correctly rounded quotient (decided here from
+    the exact rational, independently of the oracle) and agrees with the oracle
+    on every byte."""
+    from tests._quotient_points import boundary_points
+    D, Hk = 64, 2
+    pts = boundary_points(kv, 2 * Hk * D, seed=800 + kv)
+    prob, kn, vn = _problem(kv, 900 + kv, [3], [3], Hk=Hk, D=D)
+    xs = np.array([x for x, _, _ in pts], dtype=np.float64).reshape(2, Hk, D)
+    ss = np.array([s for _, s, _ in pts], dtype=np.float32).reshape(2, Hk, D)
+    want = np.array([c for _, _, c in pts]).reshape(2, Hk, D)
+    prob["k_scale"], prob["v_scale"] = ss[0].copy(), ss[1].copy()
+    kn[1] = torch.from_numpy(xs[0]).to(torch.float16)  # token 1: the boundary values
+    vn[1] = torch.from_numpy(xs[1]).to(torch.float16)
+    kc, vc, bits = _run(prob, kn, vn)
+    ko, vo = _oracle(prob, kn, vn)
+    assert bits == 0
+    np.testing.assert_array_equal(kc, ko)
+    np.testing.assert_array_equal(vc, vo)
+    bt, bs = prob["block_table"], prob["block_size"]
+    phys, slot = bt[0, 1 // bs], 1 % bs
+    for cache, w in ((kc, want[0]), (vc, want[1])):
+        row = cache[phys, slot]  # [Hk, chs]
+        if kv == KV_INT4:
+            nib = np.stack([row & 0xF, row >> 4], axis=-1).reshape(Hk, D).astype(np.int16)
+            got = np.where(nib >= 8, nib - 16, nib)
+        elif kv == KV_INT8:
+            got = row.view(np.int8).astype(np.int16)
+        else:
+            got = row.astype(np.int16)
+        np.testing.assert_array_equal(got, w)
+
+
 def test_append_bad_block_id_is_flagged_and_skipped():
     """A new token whose page id is outside the pool is not written and sets
     the BAD_BLOCK bit; the other sequences' rows are written as usual."""

@@ -292,14 +292,22 @@ def test_queries_near_bf16_max_stay_finite():
                                   "c4_ragged_prefill_int8", "c5_fp8_large_batch"])
 def test_parity_full_size_sampled(name):
     """Full workload in the launch configuration the benchmark times; the oracle
-    recomputes a sample of whole sequences (all their heads and tokens)."""
+    recomputes 16 whole sequences (all their heads and tokens; all of them when
+    the workload has fewer)."""
     w = workloads.make(name)
     out, p, ws = _gpu.run(w)
     got = out.float().cpu().double().numpy()
     rng = np.random.default_rng(2024)
     qlens = np.diff(w["cu_seqlens_q"])
     cand = np.nonzero(qlens > 0)[0]
-    seqs = rng.choice(cand, size=min(3, len(cand)), replace=False)
+    # 16 whole sequences (every one when there are fewer), always the first and
+    # the last so that both ends of the item numbering are in the sample; each
+    # sequence is checked over all of its query heads, so every KV head and
+    # head group is covered
+    pick = {int(cand[0]), int(cand[-1])}
+    rest = [int(b) for b in cand if int(b) not in pick]
+    pick.update(int(b) for b in rng.choice(rest, size=min(14, len(rest)), replace=False))
+    seqs = sorted(pick)
     cu = w["cu_seqlens_q"]
     for b in seqs:
         s = _gpu.sub_problem(w, int(b))
@@ -336,3 +344,42 @@ def test_repeated_calls_share_one_workspace():
     for o in outs[1:]:
         assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
     _check(w, outs[-1])
+
+
+@pytest.mark.parametrize("kv", ALL_KV)
+def test_full_length_beyond_the_dense_item_table(kv):
+    """300 decode sequences of up to 2048 keys: more sequences than the kernel's
+    shared-memory item table holds, so the sparse item numbering runs at full
+    lengths (with splits); 16 sampled sequences are recomputed by the oracle."""
+    B = 300
+    rng = np.random.default_rng(4242 + kv)
+    L = rng.integers(1, 2049, size=B)
+    w = workloads.make_problem(seed=4242 + kv, rng=rng, batch=B, num_heads=32, kv_num_heads=8,
+                               head_size=128, block_size=16, kv_dtype=kv, q_dtype=workloads.F16,
+                               out_dtype=workloads.F16, seqlens_k=L, q_lens=np.ones(B),
+                               pool_factor=1.0, kv_dist="fp8" if kv == KV_FP8_E4M3 else "uniform127",
+                               k_scale_range=(0.01, 0.1), v_scale_range=(0.01, 0.1),
+                               k_boost_frac=0.01)
+    out, p, ws = _gpu.run(w)
+    got = out.float().cpu().double().numpy()
+    seqs = sorted({0, B - 1} | {int(b) for b in rng.choice(np.arange(1, B - 1), 14, replace=False)})
+    for b in seqs:
+        ref = oracle.paged_attn(workloads.oracle_view(_gpu.sub_problem(w, b)))
+        vm = _gpu.vmax(w, [b])
+        assert np.max(np.abs(got[b:b + 1] - ref)) <= _gpu.TOL[0] * vm, b
+    st, bits = pa.paged_attn_read_device_error(ws)
+    assert st == pa.PA_OK and bits == 0
+
+
+def test_stream_read_checksum():
+    """The read-ceiling kernel reads every 16-byte word once: the XOR of its
+    per-block checksums equals the XOR of all words of the buffer."""
+    n = (64 << 20) + 48  # a ragged tail past the unrolled loop
+    buf = torch.randint(0, 256, (n,), dtype=torch.uint8, device="cuda")
+    sink = torch.zeros(16 * 148 * 8, dtype=torch.uint8, device="cuda")
+    pa.paged_attn_stream_read(buf, n, sink)
+    torch.cuda.synchronize()
+    words = buf.cpu().numpy().view(np.uint32).reshape(-1, 4)
+    want = np.bitwise_xor.reduce(words, axis=0)
+    got = np.bitwise_xor.reduce(sink.cpu().numpy().view(np.uint32).reshape(-1, 4), axis=0)
+    np.testing.assert_array_equal(got, want)

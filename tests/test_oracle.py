@@ -325,6 +325,19 @@ def test_quantise_ties_round_to_even_and_saturate():
     assert oracle.quantise(KV_INT8, float("nan"), s) == 0
 
 
+@pytest.mark.parametrize("kv", [KV_INT8, KV_INT4, KV_FP8_E4M3])
+def test_quantise_decides_from_the_correctly_rounded_quotient(kv):
+    """Next to a rounding boundary the code is the one nearest to the exact
+    quotient x / s (decided with rationals; every correctly rounded fp32
+    quotient lies on the same side of the boundary), at inputs where x times a
+    rounded 1 / s would give the neighbouring code."""
+    from tests._quotient_points import boundary_points
+    pts = boundary_points(kv, 48, seed=700 + kv)
+    got = [oracle.quantise(kv, x, s) for x, s, _ in pts]
+    want = [c for _, _, c in pts]
+    assert got == want
+
+
 def test_quantise_e4m3_round_trips_every_code():
     """encode(decode(c)) == c for every non-NaN code (the decode table is pinned
     by the printed code points and torch); 0x80 is the signed zero."""

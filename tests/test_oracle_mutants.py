@@ -7,7 +7,8 @@ mistake: a dropped scale, a swapped nibble, a wrong exponent bias, a wrong
 head map, an off-by-one causal limit, a transposed cache index, a flipped
 softmax sign, a wrong combine weight, a wrong fold direction; and in the
 cache writer a wrong position, a swapped nibble, truncation instead of
-rounding, a wrong INT8 range and ties to the odd e4m3 code.
+rounding, a wrong INT8 range, ties to the odd e4m3 code and a quotient
+taken as x times a rounded 1 / s instead of one correctly rounded division.
 """
 import os
 import shutil
@@ -46,6 +47,7 @@ MUTANTS = {
     "quantise_truncates": ("const float r = rintf(q);", "const float r = truncf(q);"),
     "quantise_int8_range": ("? -8 : -127;", "? -8 : -128;"),
     "e4m3_tie_odd": ("(d == best_d && (c & 1) == 0)", "(d == best_d && (c & 1) == 1)"),
+    "quantise_inverse_multiply": ("const float q = x / s;", "const float q = x * (1.0f / s);"),
 }
 
 

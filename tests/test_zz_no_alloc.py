@@ -54,3 +54,23 @@ def test_noalloc_matches_forward_on_two_calls(name, over):
         assert bool(torch.isfinite(got).all())
         err = float((got - ref.double()).abs().max())
         assert err <= tol, "no-alloc vs forward: max err %.3g > tol %.3g" % (err, tol)
+
+
+def test_noalloc_device_error_reads_back():
+    """A block-table entry outside the pool is a condition only the device sees:
+    the no-alloc call records it in its scratch's error word, which
+    paged_attn_read_device_error(NULL) returns; the next call starts clean."""
+    w = workloads.shrink("c2_int4_decode", 37, max_len=400, batch=3)
+    d = _gpu.to_device(w)
+    p, _ = _gpu.plan(w)
+    bad = d["block_table"].clone()
+    bad[1, 0] = w["num_blocks"] + 5
+    out = _new_out(w)
+    pa.paged_attn_forward_noalloc(d["q"], d["k_cache"], d["v_cache"], d["k_scale"], d["v_scale"],
+                                  bad, d["seqlens_k"], d["cu_seqlens_q"], out, p)
+    st, bits = pa.paged_attn_read_device_error(None, clear=False)
+    assert bits & pa.PA_DEVERR_BAD_BLOCK and st == pa.PA_ERR_BAD_BLOCK_TABLE
+    pa.paged_attn_forward_noalloc(d["q"], d["k_cache"], d["v_cache"], d["k_scale"], d["v_scale"],
+                                  d["block_table"], d["seqlens_k"], d["cu_seqlens_q"], out, p)
+    st, bits = pa.paged_attn_read_device_error(None)
+    assert (st, bits) == (pa.PA_OK, 0)
