@@ -16,7 +16,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libpagedattn.so")
-SOURCES = ["pa_attention.cu", "pa_codec.cu", "pa_append.cu", "pa_api.cu", "pa_noalloc.cu"]
+SOURCES = ["pa_attention.cu", "pa_prefill.cu", "pa_codec.cu", "pa_append.cu", "pa_api.cu",
+           "pa_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "-I" + INCLUDE, "-I" + CSRC]

@@ -139,9 +139,11 @@ pa_status get_encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
 }
 
 // 3-D view of one cache pool: (cache_head_size bytes, num_blocks * block_size
-// tokens, kv_num_heads); the box is 16 tokens of 4 heads, heads outermost in
-// shared memory so that each head's rows are contiguous there.
-pa_status encode_cache_map(const void* cache, const paged_attn_params* p, CUtensorMap* map) {
+// tokens, kv_num_heads); the box is 16 tokens of `box_heads` heads (4 for the
+// decode kernel, 1 for the prefill kernel), heads outermost in shared memory so
+// that each head's rows are contiguous there.
+pa_status encode_cache_map(const void* cache, const paged_attn_params* p, int box_heads,
+                           CUtensorMap* map) {
   PFN_cuTensorMapEncodeTiled_v12000 enc;
   pa_status st = get_encoder(&enc);
   if (st != PA_OK) return st;
@@ -151,8 +153,7 @@ pa_status encode_cache_map(const void* cache, const paged_attn_params* p, CUtens
                         static_cast<cuuint64_t>(p->kv_num_heads)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(chs) * p->kv_num_heads,
                            static_cast<cuuint64_t>(chs)};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(chs), 16u,
-                       static_cast<cuuint32_t>(pa::kHeadsPerItem)};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(chs), 16u, static_cast<cuuint32_t>(box_heads)};
   cuuint32_t estr[3] = {1u, 1u, 1u};
   const CUtensorMapSwizzle swz = chs == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
                                  : chs == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
@@ -215,8 +216,13 @@ pa_status paged_attn_plan(const int32_t* cu_seqlens_q_host, const int32_t* seqle
   p->max_query_len = max_q;
   p->max_seqlen_k = max_k;
   const int64_t max_rows = static_cast<int64_t>(max_q) * G;
-  // 4 rows: at most 4 rows per (sequence, KV head) (a decode step with G <= 4)
-  p->rows_per_cta = max_rows > 8 ? 16 : (max_rows > 4 ? 8 : 4);
+  // Units with more rows than one mma.sync tile (16) go to the tensor-core
+  // prefill kernel (64-row items of two KV heads) where it supports the cache
+  // format; otherwise 4 rows (at most 4 per sequence and KV head: a decode step
+  // with G <= 4), 8 or 16.
+  const bool prefill = max_rows > 16 && pa::prefill_supported(p->kv_dtype, p->head_size, bs, B);
+  p->rows_per_cta = prefill ? pa::prefill_rows_per_item()
+                            : (max_rows > 8 ? 16 : (max_rows > 4 ? 8 : 4));
   p->num_row_groups = static_cast<int>((max_rows + p->rows_per_cta - 1) / p->rows_per_cta);
   const int sms = p->num_sms > 0 ? p->num_sms : current_sm_count();
   const int max_nblk = (max_k + bs - 1) / bs;
@@ -227,14 +233,14 @@ pa_status paged_attn_plan(const int32_t* cu_seqlens_q_host, const int32_t* seqle
   // anything is split (flash decoding after the
   // GQA GEMV decode page, Code analysis 2, sized for the resident CTA slots).
   const int rows = p->rows_per_cta;
-  const int HP = pa::kHeadsPerItem;
-  const int Hg = (p->kv_num_heads + HP - 1) / HP;  // head groups: one item covers 4 KV heads
+  const int HP = prefill ? 2 : pa::kHeadsPerItem;  // KV heads per item
+  const int Hg = (p->kv_num_heads + HP - 1) / HP;  // head groups of one item each
   const double block_bytes = 2.0 * bs * cache_row_bytes(p->kv_dtype, p->head_size) *
                              (p->kv_num_heads < HP ? p->kv_num_heads : HP);
   const double item_cost = kItemCostBytes / block_bytes;
   const double part_cost = 2.0 * HP * rows * (p->head_size * 2.0 + 4.0) / block_bytes;
   const int64_t slots = static_cast<int64_t>(sms) *
-                        pa::forward_ctas_per_sm(p->kv_dtype, p->head_size, bs, rows);
+                        (prefill ? 1 : pa::forward_ctas_per_sm(p->kv_dtype, p->head_size, bs, rows));
   auto count = [&](int T, int64_t* items, int64_t* split_items, int* max_bps, int* max_ns,
                    double* work) {
     *items = *split_items = 0;
@@ -303,8 +309,11 @@ pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_c
   if (p->total_q < 0 || p->max_query_len < 0)
     return fail(PA_ERR_INVALID_ARG, "params were not filled by paged_attn_plan");
   if (p->total_q == 0 || p->batch == 0 || p->max_query_len == 0) return ok();
-  if (p->rows_per_cta != 4 && p->rows_per_cta != 8 && p->rows_per_cta != 16)
+  const bool prefill = p->rows_per_cta == pa::prefill_rows_per_item();
+  if (p->rows_per_cta != 4 && p->rows_per_cta != 8 && p->rows_per_cta != 16 && !prefill)
     return fail(PA_ERR_INVALID_ARG, "params were not filled by paged_attn_plan (rows_per_cta)");
+  if (prefill && !pa::prefill_supported(p->kv_dtype, p->head_size, p->block_size, p->batch))
+    return fail(PA_ERR_INVALID_ARG, "params were not filled by paged_attn_plan (prefill kernel)");
   if (p->rows_per_cta == 4 && p->max_query_len * (p->num_heads / p->kv_num_heads) > 4)
     return fail(PA_ERR_INVALID_ARG, "params were not filled by paged_attn_plan (rows_per_cta)");
   if (p->num_splits > kMaxSplits)
@@ -330,8 +339,9 @@ pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_c
   if (p->num_blocks == 0) return fail(PA_ERR_INVALID_ARG, "num_blocks is 0 with keys to read");
 
   CUtensorMap kmap, vmap;
-  if ((st = encode_cache_map(k_cache, p, &kmap)) != PA_OK) return st;
-  if ((st = encode_cache_map(v_cache, p, &vmap)) != PA_OK) return st;
+  const int box_heads = prefill ? 1 : pa::kHeadsPerItem;
+  if ((st = encode_cache_map(k_cache, p, box_heads, &kmap)) != PA_OK) return st;
+  if ((st = encode_cache_map(v_cache, p, box_heads, &vmap)) != PA_OK) return st;
 
   uint8_t* ws = static_cast<uint8_t*>(p->workspace);
   const WsLayout lay = ws_layout(p);
@@ -378,8 +388,9 @@ pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_c
   cudaError_t e = cudaSuccess;
   if (ev != nullptr && (e = cudaEventRecord(ev[0], s)) != cudaSuccess)
     return cuda_status(e, "profile event record");
-  e = pa::launch_forward(p->kv_dtype, p->head_size, p->block_size, p->rows_per_cta, kmap, vmap,
-                         a, s);
+  e = prefill ? pa::launch_prefill(p->block_size, kmap, vmap, a, s)
+              : pa::launch_forward(p->kv_dtype, p->head_size, p->block_size, p->rows_per_cta,
+                                   kmap, vmap, a, s);
   if (e != cudaSuccess) return cuda_status(e, "forward launch");
   if (p->num_splits > 1) {
     e = pa::launch_combine(p->head_size, p->block_size, a, s);

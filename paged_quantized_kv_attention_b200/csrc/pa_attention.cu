@@ -151,16 +151,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// One bulk copy (global -> shared) completing on an mbarrier.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
-                                          uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(dst),
-      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
-      : "memory");
-}
-
 // First of the two adjacent output dims held by accumulator elements c0 / c2 of
 // PV m-tile mt for a thread with group index g.
 template <int KV>
@@ -1453,6 +1443,7 @@ static int unit_words_t(int rows) {
 }
 
 int fragment_unit_words(int kv_dtype, int head_size, int rows_per_cta) {
+  if (rows_per_cta == prefill_rows_per_item()) return prefill_unit_words();
   const bool d128 = head_size == 128;
   switch (kv_dtype) {
     case PA_KV_INT8:

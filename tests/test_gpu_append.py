@@ -103,7 +103,8 @@ def test_append_codes_next_to_a_rounding_boundary(kv):
     on every byte."""
     from tests._quotient_points import boundary_points
     D, Hk = 64, 2
-    pts = boundary_points(kv, 2 * Hk * D, seed=800 + kv)
+    pts = boundary_points(kv, 64, seed=800 + kv)
+    pts = [pts[(i * 37) % len(pts)] for i in range(2 * Hk * D)]  # each point on several channels
     prob, kn, vn = _problem(kv, 900 + kv, [3], [3], Hk=Hk, D=D)
     xs = np.array([x for x, _, _ in pts], dtype=np.float64).reshape(2, Hk, D)
     ss = np.array([s for _, s, _ in pts], dtype=np.float32).reshape(2, Hk, D)

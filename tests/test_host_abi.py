@@ -70,7 +70,9 @@ def test_plan_zero_new_tokens_everywhere_is_a_no_op():
 def _count_items(cu, L, G, Hk, bs, rows, T, max_splits):
     """Work items by the documented split rule: a sequence with n KV blocks gets
     s = min(max_splits, ceil(n / T)) splits of ceil(n / s) blocks (empty ones
-    dropped), times its groups of 4 KV heads times its row groups."""
+    dropped), times its groups of KV heads (4 per item; 2 for the 64-row items
+    of the tensor-core prefill kernel) times its row groups."""
+    hp = 2 if rows == 64 else 4
     total, most = 0, 1
     for b in range(len(L)):
         qb = int(cu[b + 1] - cu[b])
@@ -81,7 +83,7 @@ def _count_items(cu, L, G, Hk, bs, rows, T, max_splits):
         per = -(-n // s)
         s = -(-n // per)
         most = max(most, s)
-        total += (-(-Hk // 4)) * (-(-qb * G // rows)) * s
+        total += (-(-Hk // hp)) * (-(-qb * G // rows)) * s
     return total, most
 
 
@@ -281,3 +283,28 @@ def test_noalloc_rejects_plans_beyond_its_static_scratch():
     with pytest.raises(pa.PagedAttnError) as ei:
         pa.paged_attn_forward_noalloc(*([fake] * 9), unplanned, stream=0)
     assert ei.value.status == pa.PA_ERR_INVALID_ARG
+
+
+def test_plan_sends_many_row_units_to_the_tensor_core_prefill_kernel():
+    """Units with more than 16 rows (new tokens x GQA group) over an INT8 cache
+    with head_size 128 are planned as 64-row items of the tcgen05 prefill kernel
+    (the workspace then holds one unit of query digit planes per sequence, KV
+    head and row group: 3 x 64 rows x 128 bytes and 64 multipliers); other
+    formats and shapes keep the 4/8/16-row kernel."""
+    cu = np.array([0, 16, 21], dtype=np.int32)
+    L = np.array([300, 40], dtype=np.int32)
+    for kvd, D, want in ((pa.PA_KV_INT8, 128, 64), (pa.PA_KV_INT4, 128, 16),
+                         (pa.PA_KV_FP8_E4M3, 128, 16), (pa.PA_KV_INT8, 64, 16)):
+        p = _params(batch=2, num_heads=32, kv_num_heads=8, head_size=D, block_size=16,
+                    num_blocks=64, max_blocks_per_seq=32, kv_dtype=kvd, split_blocks=-1)
+        ws = pa.paged_attn_plan(cu, L, p)
+        assert p.rows_per_cta == want, (kvd, D, p.rows_per_cta)
+        if want == 64:
+            unit = 3 * 64 * 128 + 64 * 4
+            assert p.num_row_groups == 1
+            assert ws == 256 + -(-(2 * 8 * unit) // 256) * 256  # no split here
+    # decode rows (4 per KV head) stay on the decode kernel
+    p = _params(batch=2, num_heads=32, kv_num_heads=8, head_size=128, block_size=16,
+                num_blocks=64, max_blocks_per_seq=32, kv_dtype=pa.PA_KV_INT8)
+    pa.paged_attn_plan(np.array([0, 1, 2], dtype=np.int32), L, p)
+    assert p.rows_per_cta == 4
