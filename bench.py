@@ -71,25 +71,36 @@ def algorithmic_bytes(w: dict) -> dict:
     return dict(total=total, kv=kv, qo=qo, tokens=T, fwd=total)
 
 
-def kernel_source_sha() -> str:
+# Source files of the dominant kernel of each workload (the decode kernel, or
+# the tensor-core prefill kernel for the ragged prefill workload).
+KERNEL_SOURCES = {"decode": ("pa_attention.cu", "pa_device.cuh"),
+                  "prefill": ("pa_prefill.cu", "pa_tc.cuh", "pa_device.cuh")}
+
+
+def kernel_of(name: str) -> str:
+    return "prefill" if name == "c4_ragged_prefill_int8" else "decode"
+
+
+def kernel_source_sha(kind: str = "decode") -> str:
     h = hashlib.sha256()
-    for f in ("pa_attention.cu", "pa_device.cuh"):
+    for f in KERNEL_SOURCES[kind]:
         with open(os.path.join(ROOT, "paged_quantized_kv_attention_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
 def ncu_traffic(name: str):
-    """DRAM bytes (read + write) per launch of the fused kernel from the committed
-    ncu summary profiles/ncu_traffic.txt, if it was taken on the current kernel
-    source (else None).  Line format: workload kernel_source_sha bytes_per_launch."""
+    """DRAM bytes (read + write) per launch of the workload's dominant kernel from
+    the committed ncu summary profiles/ncu_traffic.txt, if it was taken on the
+    current kernel source (else None).  Line format: workload kernel_source_sha
+    bytes_per_launch."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
     try:
         with open(path) as f:
             for ln in f:
                 parts = ln.split()
                 if len(parts) >= 3 and not ln.startswith("#") and parts[0] == name:
-                    if parts[1] == kernel_source_sha():
+                    if parts[1] == kernel_source_sha(kernel_of(name)):
                         return int(parts[2])
     except (OSError, ValueError):
         return None
@@ -145,11 +156,12 @@ def roofline_block(w: dict, ab: dict, kern_ms: float, name: str) -> dict:
     t_hbm = ab["total"] / (peak * 1e9)
     t_mma = flops / (tpk * 1e12)
     sec = kern_ms * 1e-3
+    kname = "pa_prefill_kernel" if kernel_of(name) == "prefill" else "pa_fwd_kernel"
     if t_mma > t_hbm:
-        return {"bound": "tensor", "achieved": round(flops / sec / 1e12, 2), "peak": tpk,
+        return {"bound": "tensor", "kernel": kname, "achieved": round(flops / sec / 1e12, 2), "peak": tpk,
                 "unit": "TFLOP/s", "frac": round(t_mma / sec, 4), "peak_kind": tkind,
                 "algorithmic_flops_per_launch": flops, "traffic": ncu_traffic(name)}
-    return {"bound": "hbm", "achieved": round(ab["total"] / sec / 1e9, 1), "peak": peak,
+    return {"bound": "hbm", "kernel": kname, "achieved": round(ab["total"] / sec / 1e9, 1), "peak": peak,
             "unit": "GB/s", "frac": round(t_hbm / sec, 4), "peak_kind": kind,
             "algorithmic_bytes_per_launch": ab["total"], "algorithmic_flops_per_launch": flops,
             "frac_of_tensor_peak": round(t_mma / sec, 4), "traffic": ncu_traffic(name)}
@@ -620,8 +632,8 @@ def run_ours(args):
                 "us_per_step": round(r["e2e"]["ms_per_step"] * 1e3, 2)},
         "gpu_launches": args.steps * r["launches_per_step"],
         "roofline": dict(roofline_block(r["w"], ab, r["kern_ms"], w_name),
-                         kernel="pa_fwd_kernel (timed with the other kernels of the call, "
-                                "which overlap it: the whole call on the device)",
+                         timed="the dominant kernel with the other kernels of the call, "
+                               "which overlap it: the whole call on the device",
                          kernel_us=round(r["kern_ms"] * 1e3, 3),
                          read_ceiling_gbs=ceiling["gbs_mean"] if ceiling else None),
         "read_ceiling": ceiling,

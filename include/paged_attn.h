@@ -95,7 +95,10 @@ typedef enum {
 } pa_status;
 
 typedef enum { PA_KV_INT8 = 0, PA_KV_INT4 = 1, PA_KV_FP8_E4M3 = 2 } pa_kv_dtype;
-typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
+/* Element types of q, out and the merge operands.  PA_F32 is an output type only
+ * (out of paged_attn_forward, the parts of paged_attn_merge): the unrounded rows
+ * of a partial result that another call merges. */
+typedef enum { PA_F16 = 0, PA_BF16 = 1, PA_F32 = 2 } pa_dtype;
 
 /* Bits of the device error word (see paged_attn_read_device_error). */
 #define PA_DEVERR_BAD_BLOCK 0x1u   /* block_table entry outside [0, num_blocks) */
@@ -113,8 +116,9 @@ typedef struct {
   int num_blocks;         /* physical blocks in each cache pool */
   int max_blocks_per_seq; /* columns of block_table */
   int kv_dtype;           /* pa_kv_dtype */
-  int q_dtype;            /* pa_dtype of q */
-  int out_dtype;          /* pa_dtype of out */
+  int q_dtype;            /* pa_dtype of q: PA_F16 or PA_BF16 */
+  int out_dtype;          /* pa_dtype of out: PA_F16, PA_BF16 or PA_F32 (out then
+                             16-byte aligned) */
   float softmax_scale;    /* 0 -> 1/sqrt(head_size) */
   int causal;             /* 1: bottom-right causal mask for new tokens; 0: none */
   int num_sms;            /* 0 -> SM count of the current device (148 if none) */
@@ -144,6 +148,13 @@ typedef struct {
                              cudaEvent_t that paged_attn_forward records on the
                              stream right before and right after the fused
                              attention kernel launch */
+  int stall_consumers;    /* diagnostic, 0 normally.  1: the decode kernel's
+                             consumer warps wait on a barrier that nothing
+                             signals, so that the bounded-wait path runs: the
+                             call takes about two seconds (the waits' bound),
+                             sets PA_DEVERR_TIMEOUT, leaves the output rows
+                             undefined and the GPU context usable; re-initialise
+                             the workspace before the next call. */
   float* lse_out;         /* optional: NULL, or device [total_q, num_heads] fp32
                              that receives each row's log-sum-exp of its scaled
                              logits, log sum_t exp(s_t) (natural log; -inf when the
@@ -251,15 +262,18 @@ pa_status paged_kv_unpack_int4(const uint8_t* src, int8_t* dst, int64_t rows, in
 /* Log-sum-exp merge of attention results over disjoint key sets (the flash-
  * decoding combine of the GQA GEMV decode page, Code analysis 2, across calls:
  * context parallelism, one key range per GPU).  parts: [n_parts, rows,
- * head_size] in dtype (PA_F16 / PA_BF16), each part normalised over its own
- * keys; lse_parts: [n_parts, rows] fp32, natural log, -inf for a part with no
- * key (as paged_attn_forward's lse_out gives them).  out[r] = sum_p
- * exp(lse_p[r] - lse[r]) parts[p, r] with lse[r] = log sum_p exp(lse_p[r]),
- * rounded to dtype; a row with no key in any part gets zeros.  lse_out
- * (optional, [rows]) receives lse.  1 <= n_parts <= 64; head_size 64 or 128;
- * device pointers, parts/out 8-byte aligned; async on `stream`. */
-pa_status paged_attn_merge(const void* parts, const float* lse_parts, int n_parts, int64_t rows,
-                           int head_size, int dtype, void* out, float* lse_out, void* stream);
+ * head_size] of parts_dtype (PA_F16, PA_BF16 or PA_F32), each part normalised
+ * over its own keys; lse_parts: [n_parts, rows] fp32, natural log, -inf for a
+ * part with no key (as paged_attn_forward's lse_out gives them).  out[r] =
+ * sum_p exp(lse_p[r] - lse[r]) parts[p, r] with lse[r] = log sum_p
+ * exp(lse_p[r]), accumulated in fp32 and rounded to out_dtype (PA_F16 or
+ * PA_BF16); a row with no key in any part gets zeros.  lse_out (optional,
+ * [rows]) receives lse.  1 <= n_parts <= 64; head_size 64 or 128; device
+ * pointers, parts/out 8-byte aligned (16-byte for PA_F32 parts); async on
+ * `stream`. */
+pa_status paged_attn_merge(const void* parts, int parts_dtype, const float* lse_parts,
+                           int n_parts, int64_t rows, int head_size, void* out, int out_dtype,
+                           float* lse_out, void* stream);
 
 /* Quantise-and-append: the cache write that precedes the attention call (the
  * INT4 paged-KV page, Code analysis 2-3: per-channel symmetric codes,

@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libpagedattn.so")
 PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE = 0, -1, -2, -3
 PA_ERR_BAD_BLOCK_TABLE, PA_ERR_CUDA, PA_ERR_DEVICE = -4, -5, -6
 PA_KV_INT8, PA_KV_INT4, PA_KV_FP8_E4M3 = 0, 1, 2
-PA_F16, PA_BF16 = 0, 1
+PA_F16, PA_BF16, PA_F32 = 0, 1, 2
 PA_DEVERR_BAD_BLOCK, PA_DEVERR_TIMEOUT, PA_DEVERR_BAD_SCALE, PA_DEVERR_BAD_LENGTH = 1, 2, 4, 8
 PA_NOALLOC_MAX_WORKSPACE_BYTES = 16 << 20
 
@@ -50,7 +50,7 @@ class paged_attn_params(ctypes.Structure):  # noqa: N801 (mirrors the C struct n
                 ("blocks_per_split", ctypes.c_int), ("num_work_items", ctypes.c_int),
                 ("workspace_bytes", ctypes.c_size_t),
                 ("workspace", ctypes.c_void_p), ("profile_events", ctypes.c_void_p),
-                ("lse_out", ctypes.c_void_p)]
+                ("stall_consumers", ctypes.c_int), ("lse_out", ctypes.c_void_p)]
 
 
 _lib = None
@@ -75,7 +75,7 @@ def lib() -> ctypes.CDLL:
         L.paged_kv_unpack_int4.argtypes = [P, P, ctypes.c_int64, I, P]
         L.paged_kv_gather_decode.argtypes = [P, P, PP, I, I, I, I, P, P]
         L.paged_kv_append.argtypes = [P] * 9 + [PP, P]
-        L.paged_attn_merge.argtypes = [P, P, I, ctypes.c_int64, I, I, P, P, P]
+        L.paged_attn_merge.argtypes = [P, I, P, I, ctypes.c_int64, I, P, I, P, P]
         L.paged_attn_stream_read.argtypes = [P, S, P, P]
         L.paged_attn_last_error.restype = ctypes.c_char_p
         L.paged_attn_version.restype = ctypes.c_char_p
@@ -183,11 +183,11 @@ def paged_kv_append(k_new, v_new, k_cache, v_cache, k_scale, v_scale, block_tabl
                                  _ptr(cu_seqlens_q), ctypes.byref(params), _stream(stream)))
 
 
-def paged_attn_merge(parts, lse_parts, n_parts: int, rows: int, head_size: int, dtype: int, out,
-                     lse_out=None, stream=None):
+def paged_attn_merge(parts, parts_dtype: int, lse_parts, n_parts: int, rows: int, head_size: int,
+                     out, out_dtype: int, lse_out=None, stream=None):
     """Log-sum-exp merge of results over disjoint key sets (see paged_attn.h)."""
-    _check(lib().paged_attn_merge(_ptr(parts), _ptr(lse_parts), n_parts, rows, head_size, dtype,
-                                  _ptr(out), _ptr(lse_out), _stream(stream)))
+    _check(lib().paged_attn_merge(_ptr(parts), parts_dtype, _ptr(lse_parts), n_parts, rows,
+                                  head_size, _ptr(out), out_dtype, _ptr(lse_out), _stream(stream)))
 
 
 def paged_attn_stream_read(src, nbytes: int, sink, stream=None):

@@ -1,16 +1,24 @@
 """Context parallelism: one long sequence's KV cache spread over several GPUs.
 
-Each rank holds a contiguous run of every sequence's KV blocks, runs
-``paged_attn_forward`` over its own keys with ``params.lse_out`` set, and the
-ranks exchange their (output, log-sum-exp) rows; ``paged_attn_merge`` then
-combines them exactly as the flash-decoding split of the GQA GEMV decode page
-(Code analysis 2) combines its workers' partials.  The exchange is one
-all-gather per call over ``torch.distributed`` (NCCL over NVLink on GPUs).
+Each rank holds a contiguous run of every sequence's KV blocks and runs
+``paged_attn_forward`` over its own keys with ``params.lse_out`` set and
+``out_dtype = PA_F32`` (its partial rows unrounded).  The ranks then exchange
+the rows so that each merges the rows it owns: one all-to-all of the fp32
+(output, log-sum-exp) rows, where rank r receives every rank's part of its own
+block of rows; ``paged_attn_merge`` combines them exactly as the flash-decoding
+split of the GQA GEMV decode page (Code analysis 2) combines its workers'
+partials; one all-gather of the merged rows (in the output type) gives every
+rank the whole result.  Both collectives go over ``torch.distributed`` (NCCL
+over NVLink on GPUs).  Per rank the exchange moves about T H (4 D + 4) bytes out
+and T H 2 D bytes in (T rows, H heads, head size D), independent of the rank
+count.
 
-Only new tokens that see every key of their sequence (decode, or a non-causal
-call) can be split this way: a causal new token would need the rank's key
-offset in its mask.  The helpers here are host-side plumbing; every arithmetic
-step runs in the library's kernels.
+Only new tokens that see every key of their sequence can be split this way; the
+helpers accept decode steps (at most one new token per sequence), whose token
+sees all keys.  A causal prefill row would need the rank's key offset in its
+mask, and a multi-token non-causal row would give a rank more new tokens than
+keys.  The helpers here are host-side plumbing; every arithmetic step runs in
+the library's kernels.
 """
 from __future__ import annotations
 
@@ -39,6 +47,9 @@ def local_problem(block_table, cu_seqlens_q, ranges_r, block_size: int):
     lists the global token index of every local row."""
     bt = np.asarray(block_table)
     cu = np.asarray(cu_seqlens_q, dtype=np.int64)
+    if np.any(np.diff(cu) > 1):
+        raise ValueError("context parallelism splits decode rows only: at most one new token "
+                         "per sequence (a rank's key range may be shorter than more new tokens)")
     B = bt.shape[0]
     lo, hi = ranges_r[:, 0], ranges_r[:, 1]
     nloc = (hi - lo + block_size - 1) // block_size
@@ -56,34 +67,46 @@ def local_problem(block_table, cu_seqlens_q, ranges_r, block_size: int):
     return lbt, (hi - lo).astype(np.int32), lcu, np.asarray(rows, dtype=np.int64)
 
 
-def merge_across_ranks(out_local, lse_local, rows_local, total_q: int, group=None, merge=None):
-    """All-gather every rank's rows (output [n, H, D], log-sum-exp [n, H] at
-    global token indices ``rows_local``) and merge them into [total_q, H, D].
+def merge_across_ranks(out_local, lse_local, rows_local, total_q: int, out_dtype=None,
+                       group=None, merge=None):
+    """Merge every rank's partial rows into the full result [total_q, H, D].
 
-    Rows a rank does not hold count as empty parts (log-sum-exp -inf).  ``merge``
-    defaults to the library's ``paged_attn_merge``; it is called as
-    merge(parts [W, total_q, H, D], lses [W, total_q, H], out)."""
+    ``out_local`` [n, H, D] are this rank's rows (fp32 from a forward call with
+    out_dtype PA_F32) at the global token indices ``rows_local``, ``lse_local``
+    [n, H] their log-sum-exps; rows this rank does not hold count as empty parts
+    (log-sum-exp -inf).  The rows are dealt in contiguous blocks of ceil(T / W)
+    to the W ranks: one all-to-all brings each rank every part of its block, the
+    merge combines them into ``out_dtype`` (default bf16), and one all-gather
+    returns the merged blocks to every rank.  ``merge`` defaults to the library's
+    ``paged_attn_merge``; it is called as merge(parts [W, rows, H, D],
+    lses [W, rows, H], out [rows, H, D])."""
     import torch
     import torch.distributed as dist
 
     world = dist.get_world_size(group)
     H, D = out_local.shape[1], out_local.shape[2]
-    full = out_local.new_zeros((total_q, H, D))
-    lse = torch.full((total_q, H), float("-inf"), dtype=lse_local.dtype, device=out_local.device)
+    out_dtype = out_dtype if out_dtype is not None else torch.bfloat16
+    per = -(-total_q // world)  # rows owned by each rank
+    Tp = per * world
+    dev = out_local.device
+    full = torch.zeros((Tp, H, D), dtype=out_local.dtype, device=dev)
+    lse = torch.full((Tp, H), float("-inf"), dtype=lse_local.dtype, device=dev)
     if len(rows_local):
-        idx = torch.as_tensor(rows_local, device=out_local.device)
+        idx = torch.as_tensor(rows_local, device=dev)
         full.index_copy_(0, idx, out_local)
         lse.index_copy_(0, idx, lse_local)
-    parts = [torch.empty_like(full) for _ in range(world)]
-    lses = [torch.empty_like(lse) for _ in range(world)]
-    dist.all_gather(parts, full, group=group)
-    dist.all_gather(lses, lse, group=group)
-    parts_t, lses_t = torch.stack(parts), torch.stack(lses)
-    out = torch.empty_like(full)
+    parts = torch.empty((world, per, H, D), dtype=full.dtype, device=dev)
+    lses = torch.empty((world, per, H), dtype=lse.dtype, device=dev)
+    dist.all_to_all_single(parts.view(-1), full.view(-1), group=group)
+    dist.all_to_all_single(lses.view(-1), lse.view(-1), group=group)
+    mine = torch.empty((per, H, D), dtype=out_dtype, device=dev)
     if merge is None:
-        from . import PA_BF16, PA_F16, paged_attn_merge
-        paged_attn_merge(parts_t, lses_t, world, total_q * H, D,
-                         PA_BF16 if full.dtype == torch.bfloat16 else PA_F16, out)
+        from . import PA_BF16, PA_F16, PA_F32, paged_attn_merge
+        src = {torch.float32: PA_F32, torch.bfloat16: PA_BF16, torch.float16: PA_F16}[parts.dtype]
+        paged_attn_merge(parts, src, lses, world, per * H, D, mine,
+                         PA_BF16 if out_dtype == torch.bfloat16 else PA_F16)
     else:
-        merge(parts_t, lses_t, out)
-    return out
+        merge(parts, lses, mine)
+    gathered = torch.empty((Tp, H, D), dtype=out_dtype, device=dev)
+    dist.all_gather_into_tensor(gathered, mine, group=group)
+    return gathered[:total_q]

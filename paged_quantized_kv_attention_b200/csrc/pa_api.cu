@@ -88,9 +88,10 @@ pa_status check_problem(const paged_attn_params* p) {
                 p->num_heads, p->kv_num_heads);
   if (p->kv_dtype < PA_KV_INT8 || p->kv_dtype > PA_KV_FP8_E4M3)
     return fail(PA_ERR_INVALID_ARG, "unknown kv_dtype %d", p->kv_dtype);
-  if ((p->q_dtype != PA_F16 && p->q_dtype != PA_BF16) ||
-      (p->out_dtype != PA_F16 && p->out_dtype != PA_BF16))
-    return fail(PA_ERR_INVALID_ARG, "q_dtype/out_dtype must be PA_F16 or PA_BF16");
+  if (p->q_dtype != PA_F16 && p->q_dtype != PA_BF16)
+    return fail(PA_ERR_INVALID_ARG, "q_dtype must be PA_F16 or PA_BF16");
+  if (p->out_dtype != PA_F16 && p->out_dtype != PA_BF16 && p->out_dtype != PA_F32)
+    return fail(PA_ERR_INVALID_ARG, "out_dtype must be PA_F16, PA_BF16 or PA_F32");
   if (p->head_size <= 0 || p->block_size <= 0 || p->num_blocks < 0 || p->max_blocks_per_seq < 0)
     return fail(PA_ERR_INVALID_ARG, "head_size, block_size must be > 0 and counts >= 0");
   if (p->head_size != 64 && p->head_size != 128)
@@ -102,6 +103,8 @@ pa_status check_problem(const paged_attn_params* p) {
   if (static_cast<int64_t>(p->num_blocks) * p->block_size >= (int64_t(1) << 31))
     return fail(PA_ERR_UNSUPPORTED, "num_blocks * block_size must stay below 2^31 tokens");
   if (p->causal != 0 && p->causal != 1) return fail(PA_ERR_INVALID_ARG, "causal must be 0 or 1");
+  if (p->stall_consumers != 0 && p->stall_consumers != 1)
+    return fail(PA_ERR_INVALID_ARG, "stall_consumers must be 0 or 1");
   return PA_OK;
 }
 
@@ -331,7 +334,8 @@ pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_c
     return fail(PA_ERR_INVALID_ARG, "k_cache/v_cache must be 16-byte aligned (TMA)");
   if (!aligned(q, 16) || !aligned(k_scale, 16) || !aligned(v_scale, 16))
     return fail(PA_ERR_INVALID_ARG, "q, k_scale and v_scale must be 16-byte aligned (bulk copies)");
-  if (!aligned(out, 4)) return fail(PA_ERR_INVALID_ARG, "out must be 4-byte aligned");
+  if (!aligned(out, p->out_dtype == PA_F32 ? 16 : 4))
+    return fail(PA_ERR_INVALID_ARG, "out must be 4-byte aligned (16-byte for PA_F32)");
   if (p->workspace == nullptr || p->workspace_bytes < kHeaderBytes)
     return fail(PA_ERR_WORKSPACE, "workspace missing (plan asks for %zu bytes)",
                 p->workspace_bytes);
@@ -372,6 +376,7 @@ pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_c
   a.total_q = p->total_q;
   a.q_bf16 = p->q_dtype == PA_BF16;
   a.out_bf16 = p->out_dtype == PA_BF16;
+  a.out_f32 = p->out_dtype == PA_F32;
   a.causal = p->causal;
   a.rows_cta = p->rows_per_cta;
   a.num_row_groups = p->num_row_groups;
@@ -382,6 +387,7 @@ pa_status paged_attn_forward(const void* q, const void* k_cache, const void* v_c
   const float scale = p->softmax_scale > 0.f ? p->softmax_scale
                                              : 1.0f / sqrtf(static_cast<float>(p->head_size));
   a.sm_scale_log2 = scale * 1.4426950408889634f;
+  a.stall_consumers = p->stall_consumers;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaEvent_t* ev = static_cast<cudaEvent_t*>(p->profile_events);
@@ -501,7 +507,7 @@ pa_status paged_kv_append(const void* k_new, const void* v_new, void* k_cache, v
   if (p->workspace == nullptr || p->workspace_bytes < kHeaderBytes ||
       !aligned(p->workspace, 256))
     return fail(PA_ERR_WORKSPACE, "a 256-byte aligned workspace of >= 256 bytes holds the error word");
-  if (static_cast<int64_t>(p->kv_num_heads) * p->head_size * 8 > 200 * 1024)
+  if (static_cast<int64_t>(p->kv_num_heads) * p->head_size * 16 > 200 * 1024)
     return fail(PA_ERR_UNSUPPORTED, "kv_num_heads x head_size too large for the writer's "
                 "shared-memory scales");
   pa::AppendArgs a;
@@ -526,19 +532,25 @@ pa_status paged_kv_append(const void* k_new, const void* v_new, void* k_cache, v
   return e == cudaSuccess ? ok() : cuda_status(e, "append launch");
 }
 
-pa_status paged_attn_merge(const void* parts, const float* lse_parts, int n_parts, int64_t rows,
-                           int head_size, int dtype, void* out, float* lse_out, void* stream) {
+pa_status paged_attn_merge(const void* parts, int parts_dtype, const float* lse_parts,
+                           int n_parts, int64_t rows, int head_size, void* out, int out_dtype,
+                           float* lse_out, void* stream) {
   if (!parts || !lse_parts || !out) return fail(PA_ERR_INVALID_ARG, "NULL pointer argument");
   if (n_parts < 1 || n_parts > 64) return fail(PA_ERR_INVALID_ARG, "n_parts %d not in [1, 64]", n_parts);
   if (rows < 0) return fail(PA_ERR_INVALID_ARG, "rows < 0");
   if (head_size != 64 && head_size != 128)
     return fail(PA_ERR_UNSUPPORTED, "head_size %d not in {64, 128}", head_size);
-  if (dtype != PA_F16 && dtype != PA_BF16) return fail(PA_ERR_INVALID_ARG, "dtype must be PA_F16 or PA_BF16");
-  if (!aligned(parts, 8) || !aligned(out, 8) || !aligned(lse_parts, 4))
-    return fail(PA_ERR_INVALID_ARG, "parts/out must be 8-byte and lse_parts 4-byte aligned");
+  if (parts_dtype != PA_F16 && parts_dtype != PA_BF16 && parts_dtype != PA_F32)
+    return fail(PA_ERR_INVALID_ARG, "parts_dtype must be PA_F16, PA_BF16 or PA_F32");
+  if (out_dtype != PA_F16 && out_dtype != PA_BF16)
+    return fail(PA_ERR_INVALID_ARG, "out_dtype must be PA_F16 or PA_BF16");
+  if (!aligned(parts, parts_dtype == PA_F32 ? 16 : 8) || !aligned(out, 8) || !aligned(lse_parts, 4))
+    return fail(PA_ERR_INVALID_ARG, "parts/out must be 8-byte (16 for fp32 parts) and lse_parts "
+                "4-byte aligned");
   if (rows == 0) return ok();
-  cudaError_t e = pa::launch_merge(parts, lse_parts, n_parts, rows, head_size, dtype == PA_BF16, out,
-                                   lse_out, static_cast<cudaStream_t>(stream));
+  cudaError_t e = pa::launch_merge(parts, parts_dtype, lse_parts, n_parts, rows, head_size,
+                                   out_dtype == PA_BF16, out, lse_out,
+                                   static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ok() : cuda_status(e, "merge launch");
 }
 

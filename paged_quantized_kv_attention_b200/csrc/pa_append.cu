@@ -15,7 +15,7 @@
 // handles 8-channel groups l, l + 32, ... of the token's Hk x D values (16 bytes
 // of fp16/bf16 in, 8 or 4 bytes out), so both the reads and the row writes of a
 // token (its heads are contiguous in the cache slot) are contiguous.  The
-// per-channel scales sit in shared memory.
+// per-channel scales and their rounded inverses sit in shared memory.
 //
 // Also here: the log-sum-exp merge of attention results over disjoint key sets
 // (context parallelism; the flash-decoding combine of the GQA GEMV decode page,
@@ -32,11 +32,30 @@ __device__ __forceinline__ float bits_to_float(uint32_t h, bool bf16) {
               : __half2float(__ushort_as_half(static_cast<unsigned short>(h)));
 }
 
-// Code of x under scale s: the correctly rounded fp32 quotient x / s, rounded
-// to the cache format.
+// The correctly rounded fp32 quotient x / s, given inv = 1 / s rounded to
+// nearest (or 0 when s lies outside [2^-40, 2^40]).  Markstein's correction (P.
+// Markstein, "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990): with q = RN(x inv) within one ulp
+// of x / s, the residual r = x - q s is exact in one fused multiply-add and
+// RN(q + r inv) is the correctly rounded quotient, provided nothing over- or
+// underflows, which |q| and |s| in [2^-40, 2^40] guarantee.  Elsewhere (zeros,
+// infinities, NaN, extreme operands) the quotient is taken with the correctly
+// rounded division itself.
+__device__ __forceinline__ float quotient_rn(float x, float s, float inv) {
+  const float q = __fmul_rn(x, inv);
+  const uint32_t b = __float_as_uint(q) & 0x7FFFFFFFu;
+  if (b - 0x2B800000u < 0x28000000u) {  // 2^-40 <= |q| < 2^40 (bit patterns of |q|)
+    const float r = __fmaf_rn(-q, s, x);
+    return __fmaf_rn(r, inv, q);
+  }
+  return __fdiv_rn(x, s);
+}
+
+// Code of x under scale s (inv = RN(1 / s)): the correctly rounded fp32 quotient
+// x / s, rounded to the cache format.
 template <int KV>
-__device__ __forceinline__ uint32_t code_of(float x, float s) {
-  const float q = __fdiv_rn(x, s);
+__device__ __forceinline__ uint32_t code_of(float x, float s, float inv) {
+  const float q = quotient_rn(x, s, inv);
   if constexpr (KV == PA_KV_FP8_E4M3) {
     if (q != q) return 0x7Fu;
     return static_cast<uint32_t>(__nv_cvt_float_to_fp8(q, __NV_SATFINITE, __NV_E4M3)) & 0xFFu;
@@ -52,13 +71,15 @@ __device__ __forceinline__ uint32_t code_of(float x, float s) {
 // Quantise 8 channels (16 input bytes) into their packed codes: 4 bytes (INT4)
 // or 8 bytes (INT8, FP8) in the low bits of out.
 template <int KV>
-__device__ __forceinline__ uint2 codes8(uint4 raw, float4 s0, float4 s1, bool bf16) {
+__device__ __forceinline__ uint2 codes8(uint4 raw, float4 s0, float4 s1, float4 i0, float4 i1,
+                                        bool bf16) {
   const float s[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};  // channel scales
+  const float iv[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};  // their inverses
   const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
   uint32_t c[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e)
-    c[e] = code_of<KV>(bits_to_float((w[e >> 1] >> (16 * (e & 1))) & 0xFFFFu, bf16), s[e]);
+    c[e] = code_of<KV>(bits_to_float((w[e >> 1] >> (16 * (e & 1))) & 0xFFFFu, bf16), s[e], iv[e]);
   if constexpr (KV == PA_KV_INT4) {
     uint32_t out = 0;
 #pragma unroll
@@ -80,12 +101,20 @@ __global__ void __launch_bounds__(256) pa_append_kernel(AppendArgs a) {
   constexpr int kGroups = D / 8;
   constexpr int kChs = KV == PA_KV_INT4 ? D / 2 : D;
   constexpr int kU = 4;  // groups per lane per pass (of K and of V)
-  // scales of every channel, K then V: [2][Hk][D] fp32
+  // scales of every channel, K then V, then their inverses: [2][2][Hk][D] fp32
   extern __shared__ float4 sc_s[];
   float* sc = reinterpret_cast<float*>(sc_s);
-  for (int i = threadIdx.x; i < a.Hk * D; i += blockDim.x) {
-    sc[i] = __ldg(a.k_scale + i);
-    sc[a.Hk * D + i] = __ldg(a.v_scale + i);
+  const int n = a.Hk * D;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const float ks = __ldg(a.k_scale + i), vs = __ldg(a.v_scale + i);
+    sc[i] = ks;
+    sc[n + i] = vs;
+    // the rounded inverses, 0 for a scale outside [2^-40, 2^40] (the quotient
+    // then takes the division)
+    const bool kin = fabsf(ks) >= 0x1p-40f && fabsf(ks) <= 0x1p40f;
+    const bool vin = fabsf(vs) >= 0x1p-40f && fabsf(vs) <= 0x1p40f;
+    sc[2 * n + i] = kin ? __frcp_rn(ks) : 0.f;
+    sc[3 * n + i] = vin ? __frcp_rn(vs) : 0.f;
   }
   __syncthreads();
   const int lane = threadIdx.x & 31;
@@ -134,9 +163,11 @@ __global__ void __launch_bounds__(256) pa_append_kernel(AppendArgs a) {
         if (gi >= per_tok) break;
         // channels gi * 8 .. gi * 8 + 7 of the token's Hk x D row set
         const float4* ki = sc_s + 2 * gi;
-        const float4* vi = sc_s + (a.Hk * D) / 4 + 2 * gi;
-        const uint2 kc = codes8<KV>(kr[u], ki[0], ki[1], a.in_bf16);
-        const uint2 vc = codes8<KV>(vr[u], vi[0], vi[1], a.in_bf16);
+        const float4* vi = sc_s + n / 4 + 2 * gi;
+        const float4* kinv = sc_s + n / 2 + 2 * gi;
+        const float4* vinv = sc_s + 3 * n / 4 + 2 * gi;
+        const uint2 kc = codes8<KV>(kr[u], ki[0], ki[1], kinv[0], kinv[1], a.in_bf16);
+        const uint2 vc = codes8<KV>(vr[u], vi[0], vi[1], vinv[0], vinv[1], a.in_bf16);
         // group gi is bytes [gi * 8, gi * 8 + 8) of the slot's Hk rows (INT4: 4)
         if constexpr (KV == PA_KV_INT4) {
           reinterpret_cast<uint32_t*>(kdst)[gi] = kc.x;
@@ -159,7 +190,7 @@ static cudaError_t launch_append_t(const AppendArgs& a, cudaStream_t stream) {
   const long long tasks = a.total_q;  // one warp per new token, 8 warps per CTA
   const long long want = (tasks + 7) / 8;
   const long long cap = static_cast<long long>(sms) * 8;  // 8 CTAs of 8 warps per SM
-  const size_t smem = static_cast<size_t>(a.Hk) * D * 2 * sizeof(float);
+  const size_t smem = static_cast<size_t>(a.Hk) * D * 4 * sizeof(float);
   if (smem > 48 * 1024) {
     const cudaError_t e = cudaFuncSetAttribute(pa_append_kernel<KV, D>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -188,11 +219,11 @@ cudaError_t launch_append(int kv_dtype, int head_size, const AppendArgs& a, cuda
 // ---------------------------------------------------------------------------
 // Log-sum-exp merge of results over disjoint key sets: one warp per row; lane p
 // holds part p's weight (n_parts <= 64: two per lane), then each lane sums its
-// dims over the parts.
-template <int D>
-__global__ void __launch_bounds__(128) pa_merge_kernel(const uint16_t* __restrict__ parts,
+// dims (a pair per step) over the parts in fp32.  PT: the parts' element type.
+template <int D, int PT>
+__global__ void __launch_bounds__(128) pa_merge_kernel(const void* __restrict__ parts,
                                                        const float* __restrict__ lse_parts,
-                                                       int n_parts, long long rows, bool bf16,
+                                                       int n_parts, long long rows, bool out_bf16,
                                                        uint16_t* __restrict__ out,
                                                        float* __restrict__ lse_out) {
   const int lane = threadIdx.x & 31;
@@ -211,21 +242,33 @@ __global__ void __launch_bounds__(128) pa_merge_kernel(const uint16_t* __restric
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   const float inv = sum > 0.f ? 1.f / sum : 0.f;
   if (lse_out != nullptr && lane == 0) lse_out[r] = sum > 0.f ? M + __logf(sum) : -INFINITY;
-  constexpr int kPairs = D / 2;  // half2 pairs per row
+  constexpr int kPairs = D / 2;  // element pairs per row
   for (int d2 = lane; d2 < kPairs; d2 += 32) {
     float ax = 0.f, ay = 0.f;
     for (int pidx = 0; pidx < n_parts; ++pidx) {
       const float wv = __shfl_sync(0xffffffffu, pidx < 32 ? w0 : w1, pidx & 31) * inv;
       if (wv == 0.f) continue;  // empty part: its values are not read
-      const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(
-          parts + (static_cast<long long>(pidx) * rows + r) * D) + d2);
-      const float x = bf16 ? __uint_as_float(v << 16) : __half2float(__ushort_as_half(v & 0xFFFFu));
-      const float y = bf16 ? __uint_as_float(v & 0xFFFF0000u) : __half2float(__ushort_as_half(v >> 16));
+      const long long e = (static_cast<long long>(pidx) * rows + r) * D;  // row start, elements
+      float x, y;
+      if constexpr (PT == PA_F32) {
+        const float2 v = __ldg(reinterpret_cast<const float2*>(static_cast<const float*>(parts) + e) + d2);
+        x = v.x;
+        y = v.y;
+      } else {
+        const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(static_cast<const uint16_t*>(parts) + e) + d2);
+        if constexpr (PT == PA_BF16) {
+          x = __uint_as_float(v << 16);
+          y = __uint_as_float(v & 0xFFFF0000u);
+        } else {
+          x = __half2float(__ushort_as_half(v & 0xFFFFu));
+          y = __half2float(__ushort_as_half(v >> 16));
+        }
+      }
       ax = fmaf(wv, x, ax);
       ay = fmaf(wv, y, ay);
     }
     uint32_t o;
-    if (bf16) {
+    if (out_bf16) {
       const __nv_bfloat162 h = __floats2bfloat162_rn(ax, ay);
       o = *reinterpret_cast<const uint32_t*>(&h);
     } else {
@@ -236,20 +279,38 @@ __global__ void __launch_bounds__(128) pa_merge_kernel(const uint16_t* __restric
   }
 }
 
-cudaError_t launch_merge(const void* parts, const float* lse_parts, int n_parts, long long rows,
-                         int head_size, bool bf16, void* out, float* lse_out, cudaStream_t stream) {
+template <int D>
+static cudaError_t launch_merge_d(const void* parts, int parts_dtype, const float* lse_parts,
+                                  int n_parts, long long rows, bool out_bf16, uint16_t* out,
+                                  float* lse_out, unsigned blocks, cudaStream_t stream) {
+  switch (parts_dtype) {
+    case PA_F32:
+      pa_merge_kernel<D, PA_F32><<<blocks, 128, 0, stream>>>(parts, lse_parts, n_parts, rows,
+                                                             out_bf16, out, lse_out);
+      break;
+    case PA_BF16:
+      pa_merge_kernel<D, PA_BF16><<<blocks, 128, 0, stream>>>(parts, lse_parts, n_parts, rows,
+                                                              out_bf16, out, lse_out);
+      break;
+    default:
+      pa_merge_kernel<D, PA_F16><<<blocks, 128, 0, stream>>>(parts, lse_parts, n_parts, rows,
+                                                             out_bf16, out, lse_out);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge(const void* parts, int parts_dtype, const float* lse_parts, int n_parts,
+                         long long rows, int head_size, bool out_bf16, void* out, float* lse_out,
+                         cudaStream_t stream) {
   if (rows <= 0) return cudaSuccess;
   const long long blocks = (rows + 3) / 4;
   if (blocks >= (1ll << 31)) return cudaErrorInvalidValue;
-  const auto* pp = static_cast<const uint16_t*>(parts);
   auto* op = static_cast<uint16_t*>(out);
   if (head_size == 128)
-    pa_merge_kernel<128><<<static_cast<unsigned>(blocks), 128, 0, stream>>>(pp, lse_parts, n_parts,
-                                                                            rows, bf16, op, lse_out);
-  else
-    pa_merge_kernel<64><<<static_cast<unsigned>(blocks), 128, 0, stream>>>(pp, lse_parts, n_parts,
-                                                                           rows, bf16, op, lse_out);
-  return cudaGetLastError();
+    return launch_merge_d<128>(parts, parts_dtype, lse_parts, n_parts, rows, out_bf16, op, lse_out,
+                               static_cast<unsigned>(blocks), stream);
+  return launch_merge_d<64>(parts, parts_dtype, lse_parts, n_parts, rows, out_bf16, op, lse_out,
+                            static_cast<unsigned>(blocks), stream);
 }
 
 }  // namespace pa

@@ -113,7 +113,9 @@ struct Cfg {
   static constexpr int kStages = kStagesRaw > 32 ? 32 : (kStagesRaw < 2 ? 2 : kStagesRaw);
   static constexpr int kRingBytes = kStages * kStageBytes;
   static constexpr int kBarOff = kRingBytes;
-  static constexpr int kNumBars = 2 * kStages + 5;  // full, empty, item full/empty x2, fragments
+  // full, empty, item full/empty x2, fragments, and one that is never signalled
+  // (the stall_consumers diagnostic)
+  static constexpr int kNumBars = 2 * kStages + 6;
   static constexpr int kDescOff = kBarOff + kNumBars * 8;
   // the producer's item table: inclusive item prefix per sequence, for as many
   // sequences (a multiple of 32, at most 256) as the budget leaves room for
@@ -469,6 +471,8 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
   auto item_empty = [&](int sl) { return smem_u32(bars + 2 * C::kStages + 2 + sl); };
   // completes once every consumer warp holds its first item's query fragments
   const uint32_t frag_ready = smem_u32(bars + 2 * C::kStages + 4);
+  // never completes: the consumers of a stall_consumers call wait on it
+  const uint32_t never_bar = smem_u32(bars + 2 * C::kStages + 5);
   auto k_tile = [&](int s) { return smem + s * C::kStageBytes; };
   auto v_tile = [&](int s) { return smem + s * C::kStageBytes + C::kKTile; };
 
@@ -496,6 +500,7 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
       mbar_init(item_empty(lane), C::kWarps);
     }
     if (lane == 2) mbar_init(frag_ready, C::kWarps);
+    if (lane == 3) mbar_init(never_bar, 1);
     mbar_fence_init();
   }
   __syncthreads();
@@ -764,6 +769,13 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
     if (!prep_done) {
       asm volatile("griddepcontrol.wait;" ::: "memory");
       prep_done = true;
+      // Diagnostic: a wait that nothing ends.  Its bound runs out, the warp
+      // records the timeout and leaves; the producer's own bounded waits then
+      // run out too and it drains every copy it issued before the CTA exits.
+      if (a.stall_consumers && !mbar_wait(never_bar, 0)) {
+        if (lane == 0) record_error(a.err, PA_DEVERR_TIMEOUT);
+        return;
+      }
     }
     uint32_t qf[NT][C::kQWords];
     float wA[NT][2], wB[NT][2];
@@ -1170,7 +1182,10 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, NT, LP>::kThreads) __maxnreg__(
               const float2 vs = __ldg(reinterpret_cast<const float2*>(vsc + dd));
               const float o0 = o[nt][mt][j] * inv * vs.x;
               const float o1 = o[nt][mt][j + 2] * inv * vs.y;
-              if (a.out_bf16)
+              if (a.out_f32)
+                *reinterpret_cast<float2*>(reinterpret_cast<float*>(a.out) + orow * D + dd) =
+                    make_float2(o0, o1);
+              else if (a.out_bf16)
                 *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(a.out) +
                                                    orow * D + dd) = __floats2bfloat162_rn(o0, o1);
               else
@@ -1317,7 +1332,9 @@ __global__ void __launch_bounds__(128) pa_combine_kernel(const FwdArgs a) {
   acc.z *= vs.z;
   acc.w *= vs.w;
   const size_t o = static_cast<size_t>(gr) * D + 4 * lane;
-  if (a.out_bf16) {
+  if (a.out_f32) {
+    *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + o) = acc;
+  } else if (a.out_bf16) {
     __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(a.out) + o);
     dst[0] = __floats2bfloat162_rn(acc.x, acc.y);
     dst[1] = __floats2bfloat162_rn(acc.z, acc.w);

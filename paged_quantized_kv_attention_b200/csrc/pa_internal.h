@@ -27,7 +27,7 @@ struct FwdArgs {
   uint32_t* work;       // [2]: next work item, CTAs finished (both rewound by the last CTA)
   uint32_t* err;        // sticky device error word
   int batch, H, Hk, G, maxb, num_blocks, total_q;
-  int q_bf16, out_bf16, causal;
+  int q_bf16, out_bf16, out_f32, causal;  // out_f32: fp32 rows (for a later merge)
   int rows_cta;         // query rows per (KV head, row group): 4, 8 or 16
   int num_row_groups;   // largest number of row groups of a (sequence, KV head)
   int max_splits;       // partial slots: no sequence is split into more items
@@ -36,6 +36,7 @@ struct FwdArgs {
   int num_items;        // work items of the plan (grid = min(num_items, resident CTAs))
   int num_sms;          // SMs of the device
   float sm_scale_log2;  // softmax_scale * log2(e)
+  int stall_consumers;  // diagnostic: consumer warps wait on a barrier nothing signals
 };
 
 // KV heads of one work item: the fused kernel streams their rows of a block with
@@ -78,8 +79,9 @@ struct AppendArgs {
 };
 cudaError_t launch_append(int kv_dtype, int head_size, const AppendArgs& a, cudaStream_t stream);
 // Log-sum-exp merge of results over disjoint key sets (pa_append.cu).
-cudaError_t launch_merge(const void* parts, const float* lse_parts, int n_parts, long long rows,
-                         int head_size, bool bf16, void* out, float* lse_out, cudaStream_t stream);
+cudaError_t launch_merge(const void* parts, int parts_dtype, const float* lse_parts, int n_parts,
+                         long long rows, int head_size, bool out_bf16, void* out, float* lse_out,
+                         cudaStream_t stream);
 
 // Launcher (pa_attention.cu).  rows_per_cta is 4 (decode rows packed with their
 // fp16 residuals), 8 or 16.

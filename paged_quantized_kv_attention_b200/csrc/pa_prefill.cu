@@ -880,7 +880,17 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           tmem_wait_ld();
           if (!valid) continue;
           uint32_t packed[8];
-          if (!is_split) {
+          if (!is_split && a.out_f32) {
+            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + orow * kPfD + 16 * c);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float4 vs = reinterpret_cast<const float4*>(vsc + 16 * c)[j];
+              dst[j] = make_float4(__uint_as_float(o[4 * j]) * inv * vs.x,
+                                   __uint_as_float(o[4 * j + 1]) * inv * vs.y,
+                                   __uint_as_float(o[4 * j + 2]) * inv * vs.z,
+                                   __uint_as_float(o[4 * j + 3]) * inv * vs.w);
+            }
+          } else if (!is_split) {
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
               const float2 vs = reinterpret_cast<const float2*>(vsc + 16 * c)[j];

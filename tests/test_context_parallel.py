@@ -84,7 +84,8 @@ def _gloo_rank(rank, world, port, result):
         out.copy_(torch.from_numpy(m.reshape(T, H, D)))
 
     T = int(prob["cu_seqlens_q"][-1])
-    out = cp.merge_across_ranks(torch.from_numpy(o), torch.from_numpy(lse), rows, T, merge=merge)
+    out = cp.merge_across_ranks(torch.from_numpy(o), torch.from_numpy(lse), rows, T,
+                                out_dtype=torch.float64, merge=merge)
     if rank == 0:
         ref = oracle.paged_attn(prob)
         result.put(float(np.max(np.abs(out.numpy() - ref)) / np.max(np.abs(ref))))
@@ -93,8 +94,9 @@ def _gloo_rank(rank, world, port, result):
 
 
 def test_gloo_two_ranks_merge_to_the_unsplit_result():
-    """World size 2 over gloo: shards, gather order and merge give the oracle's
-    unsplit attention (1e-12)."""
+    """World size 2 over gloo: shards, the all-to-all of each rank's rows to their
+    owners, the merge and the all-gather give the oracle's unsplit attention
+    (1e-12)."""
     import torch.multiprocessing as mp
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
@@ -118,8 +120,8 @@ def _gpu_forward(w, lse=True, **over):
     ws = torch.zeros(max(nb, 256), dtype=torch.uint8, device="cuda")
     p.workspace = ws.data_ptr()
     T, H, D = int(w["cu_seqlens_q"][-1]), w["num_heads"], w["head_size"]
-    out = torch.empty((T, H, D), dtype=torch.bfloat16 if w["out_dtype"] else torch.float16,
-                      device="cuda")
+    odt = {0: torch.float16, 1: torch.bfloat16, 2: torch.float32}[w["out_dtype"]]
+    out = torch.empty((T, H, D), dtype=odt, device="cuda")
     lse_t = torch.empty((T, H), dtype=torch.float32, device="cuda")
     if lse:
         p.lse_out = lse_t.data_ptr()
@@ -165,9 +167,10 @@ def test_rank_local_calls_merge_to_the_full_result(kv, world):
     from tests import _gpu
     prob = _problem(20 + kv + world, kv=kv)
     w = _as_w(prob)
+    w["out_dtype"] = pa.PA_F32  # the ranks' partial rows, unrounded
     T, H, D = int(w["cu_seqlens_q"][-1]), w["num_heads"], w["head_size"]
     ranges = cp.shard_ranges(prob["seqlens_k"], prob["block_size"], world)
-    parts = torch.zeros((world, T, H, D), dtype=torch.bfloat16, device="cuda")
+    parts = torch.zeros((world, T, H, D), dtype=torch.float32, device="cuda")
     lses = torch.full((world, T, H), float("-inf"), dtype=torch.float32, device="cuda")
     for r in range(world):
         lbt, lL, lcu, rows = cp.local_problem(prob["block_table"], prob["cu_seqlens_q"], ranges[r],
@@ -181,8 +184,36 @@ def test_rank_local_calls_merge_to_the_full_result(kv, world):
         parts[r].index_copy_(0, idx, o)
         lses[r].index_copy_(0, idx, l)
     out = torch.empty((T, H, D), dtype=torch.bfloat16, device="cuda")
-    pa.paged_attn_merge(parts, lses, world, T * H, D, pa.PA_BF16, out)
+    pa.paged_attn_merge(parts, pa.PA_F32, lses, world, T * H, D, out, pa.PA_BF16)
     torch.cuda.synchronize()
     ref = oracle.paged_attn(workloads.oracle_view(w))
     got = out.double().cpu().numpy()
     assert np.max(np.abs(got - ref)) <= _gpu.TOL[1] * _gpu.vmax(w)
+
+
+def test_local_problem_is_for_decode_rows_only():
+    """A rank's key range can be shorter than a sequence's new tokens, so only
+    decode steps (at most one new token per sequence) are split across ranks."""
+    prob = _problem(7)
+    ranges = cp.shard_ranges(prob["seqlens_k"], prob["block_size"], 2)
+    cu = np.array([0, 1, 3, 4, 5], dtype=np.int32)  # sequence 1 has two new tokens
+    with pytest.raises(ValueError):
+        cp.local_problem(prob["block_table"], cu, ranges[0], prob["block_size"])
+
+
+@pytest.mark.gpu
+def test_fp32_output_matches_the_rounded_one():
+    """out_dtype PA_F32 gives the unrounded rows: rounding them to bf16 gives the
+    bf16 call's output to within one bf16 rounding, and both meet the bar."""
+    from tests import _gpu
+    prob = _problem(31)
+    w = _as_w(prob)
+    o16, _, _ = _gpu_forward(w)
+    w32 = dict(w, out_dtype=pa.PA_F32)
+    o32, _, _ = _gpu_forward(w32)
+    assert o32.dtype == torch.float32
+    ref = oracle.paged_attn(workloads.oracle_view(w))
+    vm = _gpu.vmax(w)
+    assert np.max(np.abs(o32.double().cpu().numpy() - ref)) <= _gpu.TOL[0] * vm
+    diff = (o32.to(torch.bfloat16).float() - o16.float()).abs().max().item()
+    assert diff <= 2 ** -7 * vm

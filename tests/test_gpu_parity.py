@@ -383,3 +383,31 @@ def test_stream_read_checksum():
     want = np.bitwise_xor.reduce(words, axis=0)
     got = np.bitwise_xor.reduce(sink.cpu().numpy().view(np.uint32).reshape(-1, 4), axis=0)
     np.testing.assert_array_equal(got, want)
+
+
+def test_bounded_wait_runs_out_and_the_context_stays_usable():
+    """The consumer warps wait on a barrier that nothing signals (the
+    stall_consumers diagnostic): the wait's bound runs out, the kernel records
+    PA_DEVERR_TIMEOUT and returns (its producer drains every copy it issued), and
+    the next call on the re-initialised workspace is correct."""
+    w = workloads.shrink("c2_int4_decode", 41, max_len=300, batch=3)
+    d = _gpu.to_device(w)
+    p, nb = _gpu.plan(w, split_blocks=-1)
+    ws = torch.empty(max(nb, 256), dtype=torch.uint8, device="cuda")
+    pa.paged_attn_workspace_init(ws, ws.numel())
+    p.workspace = ws.data_ptr()
+    p.stall_consumers = 1
+    out = torch.empty((int(w["cu_seqlens_q"][-1]), w["num_heads"], w["head_size"]),
+                      dtype=torch.float16, device="cuda")
+    pa.paged_attn_forward(d["q"], d["k_cache"], d["v_cache"], d["k_scale"], d["v_scale"],
+                          d["block_table"], d["seqlens_k"], d["cu_seqlens_q"], out, p)
+    torch.cuda.synchronize()
+    st, bits = pa.paged_attn_read_device_error(ws)
+    assert bits & pa.PA_DEVERR_TIMEOUT and st == pa.PA_ERR_DEVICE
+    p.stall_consumers = 0
+    pa.paged_attn_workspace_init(ws, ws.numel())
+    pa.paged_attn_forward(d["q"], d["k_cache"], d["v_cache"], d["k_scale"], d["v_scale"],
+                          d["block_table"], d["seqlens_k"], d["cu_seqlens_q"], out, p)
+    torch.cuda.synchronize()
+    assert pa.paged_attn_read_device_error(ws) == (pa.PA_OK, 0)
+    _check(w, out)

@@ -231,15 +231,28 @@ def test_append_checks_arguments_before_any_launch():
 def test_merge_checks_arguments_before_any_launch():
     buf = np.zeros(1024, dtype=np.uint8)
     al = buf[(-buf.ctypes.data) % 16:]
-    for bad in (dict(n_parts=0), dict(n_parts=65), dict(head_size=96), dict(dtype=7)):
-        kw = dict(n_parts=2, head_size=128, dtype=pa.PA_F16)
+    for bad in (dict(n_parts=0), dict(n_parts=65), dict(head_size=96), dict(src=7),
+                dict(dst=pa.PA_F32), dict(dst=7)):
+        kw = dict(n_parts=2, head_size=128, src=pa.PA_F32, dst=pa.PA_F16)
         kw.update(bad)
         with pytest.raises(pa.PagedAttnError):
-            pa.paged_attn_merge(al, al, kw["n_parts"], 4, kw["head_size"], kw["dtype"], al, stream=0)
+            pa.paged_attn_merge(al, kw["src"], al, kw["n_parts"], 4, kw["head_size"], al, kw["dst"],
+                                stream=0)
     with pytest.raises(pa.PagedAttnError) as ei:
-        pa.paged_attn_merge(None, al, 2, 4, 128, pa.PA_F16, al, stream=0)
+        pa.paged_attn_merge(None, pa.PA_F16, al, 2, 4, 128, al, pa.PA_F16, stream=0)
     assert ei.value.status == pa.PA_ERR_INVALID_ARG
-    pa.paged_attn_merge(al, al, 2, 0, 128, pa.PA_F16, al, stream=0)  # no rows: nothing launched
+    with pytest.raises(pa.PagedAttnError):  # fp32 parts must be 16-byte aligned
+        pa.paged_attn_merge(al[8:], pa.PA_F32, al, 2, 4, 128, al, pa.PA_F16, stream=0)
+    pa.paged_attn_merge(al, pa.PA_F32, al, 2, 0, 128, al, pa.PA_F16, stream=0)  # no rows: no launch
+
+
+def test_forward_accepts_fp32_output_and_rejects_it_for_queries():
+    p = _params(out_dtype=pa.PA_F32)
+    pa.paged_attn_plan(np.array([0, 1, 2, 3, 4], dtype=np.int32), np.array([40, 5, 9, 100]), p)
+    p = _params(q_dtype=pa.PA_F32)
+    with pytest.raises(pa.PagedAttnError) as ei:
+        pa.paged_attn_plan(np.array([0, 1, 2, 3, 4], dtype=np.int32), np.array([40, 5, 9, 100]), p)
+    assert ei.value.status == pa.PA_ERR_INVALID_ARG
 
 
 def test_codec_entry_points_check_arguments():
