@@ -32,44 +32,37 @@ __device__ __forceinline__ float bits_to_float(uint32_t h, bool bf16) {
               : __half2float(__ushort_as_half(static_cast<unsigned short>(h)));
 }
 
-// The correctly rounded fp32 quotient x / s, given inv = 1 / s rounded to
-// nearest (or 0 when s lies outside [2^-40, 2^40]).  Markstein's correction (P.
-// Markstein, "Computation of elementary functions on the IBM RISC System/6000
-// processor", IBM J. Res. Dev. 34(1), 1990): with q = RN(x inv) within one ulp
-// of x / s, the residual r = x - q s is exact in one fused multiply-add and
-// RN(q + r inv) is the correctly rounded quotient, provided nothing over- or
-// underflows, which |q| and |s| in [2^-40, 2^40] guarantee.  Elsewhere (zeros,
-// infinities, NaN, extreme operands) the quotient is taken with the correctly
-// rounded division itself.
-__device__ __forceinline__ float quotient_rn(float x, float s, float inv) {
-  const float q = __fmul_rn(x, inv);
-  const uint32_t b = __float_as_uint(q) & 0x7FFFFFFFu;
-  if (b - 0x2B800000u < 0x28000000u) {  // 2^-40 <= |q| < 2^40 (bit patterns of |q|)
-    const float r = __fmaf_rn(-q, s, x);
-    return __fmaf_rn(r, inv, q);
-  }
-  return __fdiv_rn(x, s);
-}
+// Code of x under scale s (inv = RN(1 / s)): the code of the correctly rounded
+// fp32 quotient x / s.  Integer caches: x * inv is within 2^-16 of x / s for
+// |x / s| < 128 (two roundings of 2^-24 relative each), so its nearest integer
+// is the code unless it lies within 2^-15 of a half-integer boundary (or on
+// one); only then is the correctly rounded division taken.  Beyond the code
+// range both forms clamp alike.  FP8: the correctly rounded division.
+// The correctly rounded division, out of line: it runs only near a rounding
+// boundary, and a call keeps it off the path of every other value.
+__device__ __noinline__ float div_rn(float x, float s) { return __fdiv_rn(x, s); }
 
-// Code of x under scale s (inv = RN(1 / s)): the correctly rounded fp32 quotient
-// x / s, rounded to the cache format.
 template <int KV>
 __device__ __forceinline__ uint32_t code_of(float x, float s, float inv) {
-  const float q = quotient_rn(x, s, inv);
   if constexpr (KV == PA_KV_FP8_E4M3) {
+    const float q = __fdiv_rn(x, s);
     if (q != q) return 0x7Fu;
     return static_cast<uint32_t>(__nv_cvt_float_to_fp8(q, __NV_SATFINITE, __NV_E4M3)) & 0xFFu;
   } else {
-    if (q != q) return 0u;
-    constexpr float lo = KV == PA_KV_INT4 ? -8.f : -127.f;
-    constexpr float hi = KV == PA_KV_INT4 ? 7.f : 127.f;
-    const float r = fminf(fmaxf(rintf(q), lo), hi);
-    return static_cast<uint32_t>(static_cast<int>(r)) & (KV == PA_KV_INT4 ? 0xFu : 0xFFu);
+    float q = __fmul_rn(x, inv);
+    float r = rintf(q);
+    if (__builtin_expect(fabsf(q - r) > 0.5f - 0x1p-15f, 0)) {
+      q = div_rn(x, s);
+      r = rintf(q);
+    }
+    // nearest integer, clamped (a NaN quotient converts to 0)
+    constexpr int lo = KV == PA_KV_INT4 ? -8 : -127;
+    constexpr int hi = KV == PA_KV_INT4 ? 7 : 127;
+    const int c = min(max(__float2int_rn(r), lo), hi);
+    return static_cast<uint32_t>(c) & (KV == PA_KV_INT4 ? 0xFu : 0xFFu);
   }
 }
 
-// Quantise 8 channels (16 input bytes) into their packed codes: 4 bytes (INT4)
-// or 8 bytes (INT8, FP8) in the low bits of out.
 template <int KV>
 __device__ __forceinline__ uint2 codes8(uint4 raw, float4 s0, float4 s1, float4 i0, float4 i1,
                                         bool bf16) {
@@ -109,12 +102,8 @@ __global__ void __launch_bounds__(256) pa_append_kernel(AppendArgs a) {
     const float ks = __ldg(a.k_scale + i), vs = __ldg(a.v_scale + i);
     sc[i] = ks;
     sc[n + i] = vs;
-    // the rounded inverses, 0 for a scale outside [2^-40, 2^40] (the quotient
-    // then takes the division)
-    const bool kin = fabsf(ks) >= 0x1p-40f && fabsf(ks) <= 0x1p40f;
-    const bool vin = fabsf(vs) >= 0x1p-40f && fabsf(vs) <= 0x1p40f;
-    sc[2 * n + i] = kin ? __frcp_rn(ks) : 0.f;
-    sc[3 * n + i] = vin ? __frcp_rn(vs) : 0.f;
+    sc[2 * n + i] = __frcp_rn(ks);  // the rounded inverses
+    sc[3 * n + i] = __frcp_rn(vs);
   }
   __syncthreads();
   const int lane = threadIdx.x & 31;
