@@ -220,9 +220,9 @@ pa_status paged_attn_plan(const int32_t* cu_seqlens_q_host, const int32_t* seqle
   p->max_seqlen_k = max_k;
   const int64_t max_rows = static_cast<int64_t>(max_q) * G;
   // Units with more rows than one mma.sync tile (16) go to the tensor-core
-  // prefill kernel (64-row items of two KV heads) where it supports the cache
-  // format; otherwise 4 rows (at most 4 per sequence and KV head: a decode step
-  // with G <= 4), 8 or 16.
+  // prefill kernel (items of one KV head and up to 64 rows) where it supports
+  // the cache format; otherwise 4 rows (at most 4 per sequence and KV head: a
+  // decode step with G <= 4), 8 or 16.
   const bool prefill = max_rows > 16 && pa::prefill_supported(p->kv_dtype, p->head_size, bs, B);
   p->rows_per_cta = prefill ? pa::prefill_rows_per_item()
                             : (max_rows > 8 ? 16 : (max_rows > 4 ? 8 : 4));
@@ -236,7 +236,7 @@ pa_status paged_attn_plan(const int32_t* cu_seqlens_q_host, const int32_t* seqle
   // anything is split (flash decoding after the
   // GQA GEMV decode page, Code analysis 2, sized for the resident CTA slots).
   const int rows = p->rows_per_cta;
-  const int HP = prefill ? 2 : pa::kHeadsPerItem;  // KV heads per item
+  const int HP = prefill ? 1 : pa::kHeadsPerItem;  // KV heads per item
   const int Hg = (p->kv_num_heads + HP - 1) / HP;  // head groups of one item each
   const double block_bytes = 2.0 * bs * cache_row_bytes(p->kv_dtype, p->head_size) *
                              (p->kv_num_heads < HP ? p->kv_num_heads : HP);

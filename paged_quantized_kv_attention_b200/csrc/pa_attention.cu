@@ -1352,6 +1352,21 @@ template <int D, int BS>
 static cudaError_t launch_combine_t(const FwdArgs& a, cudaStream_t stream) {
   const long long rows = static_cast<long long>(a.total_q) * a.H;
   if (rows <= 0) return cudaSuccess;
+  // Like the forward kernels, the combine prefers the largest shared-memory
+  // carveout, so that no SM is reconfigured between the kernels of a call.
+  static std::atomic<int> configured[64] = {};
+  int dev = 0;
+  cudaError_t ce = cudaGetDevice(&dev);
+  if (ce != cudaSuccess) return ce;
+  if (dev >= 64 || !configured[dev].load(std::memory_order_acquire)) {
+    ce = cudaFuncSetAttribute(pa_combine_kernel<D, BS, 1>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                              cudaSharedmemCarveoutMaxShared);
+    if (ce != cudaSuccess) return ce;
+    ce = cudaFuncSetAttribute(pa_combine_kernel<D, BS, 4>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                              cudaSharedmemCarveoutMaxShared);
+    if (ce != cudaSuccess) return ce;
+    if (dev < 64) configured[dev].store(1, std::memory_order_release);
+  }
   const bool few = rows < kCombineSplitWarpRows;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(few ? rows : (rows + 3) / 4));

@@ -91,9 +91,9 @@ cudaError_t launch_forward(int kv_dtype, int head_size, int block_size, int rows
 // Log-sum-exp merge of the split partials (one warp per row of a split unit),
 // launched right after the forward kernel as its programmatic dependent.
 cudaError_t launch_combine(int head_size, int block_size, const FwdArgs& a, cudaStream_t stream);
-// Tensor-core prefill kernel (pa_prefill.cu): work items of 64 query rows of
-// two KV heads.  Supported for INT8 caches, head_size 128, block_size 16 or 32,
-// batch <= 1024.
+// Tensor-core prefill kernel (pa_prefill.cu): work items of up to 64 query rows
+// of one KV head.  Supported for INT8 caches, head_size 128, block_size 16 or
+// 32, batch <= 1024.
 bool prefill_supported(int kv_dtype, int head_size, int block_size, int batch);
 int prefill_rows_per_item();
 // 32-bit words of one (sequence, KV head, row group) unit of query digits in

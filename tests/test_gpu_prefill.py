@@ -3,11 +3,12 @@ against the FP64 oracle, through the C ABI.
 
 The planner sends units with more than 16 query rows per KV head (new tokens x
 GQA group) over an INT8 cache with head_size 128 to this kernel (work items of
-64 rows of two KV heads).  Cases: ragged causal prefill with zero-new-token
-sequences, lengths on and off the 64-key tile and the 16/32-token block edges,
-more than one row group, forced KV splits (the combine kernel), an odd KV head
-count (a pair with one head), non-causal calls, bf16 queries and output, the
-per-row log-sum-exp, extreme K scales, a bad block id.  Tolerance as for the
+one KV head and up to 64 rows, padded to 16, 32, 48 or 64; 128-key tiles).
+Cases: ragged causal prefill with zero-new-token sequences, every row padding,
+lengths on and off the 128-key tile and the 16/32-token block edges, more than
+one row group, forced KV splits (the combine kernel), an odd KV head count,
+non-causal calls, bf16 queries and output, fp32 output, the per-row
+log-sum-exp, extreme K scales, a bad block id.  Tolerance as for the
 decode path: max|out - ref| <= 2e-3 * max|dequant(V)| (fp16 out), 8e-3 (bf16).
 """
 import numpy as np
@@ -81,7 +82,7 @@ def test_forced_splits_merge_in_the_combine(split_blocks):
 
 
 def test_odd_kv_head_count():
-    """Hk = 3: the last item pair holds one KV head."""
+    """Hk = 3, G = 8: 24 query heads."""
     rng = np.random.default_rng(630)
     prob, _ = paged_problem(rng, kv_dtype=KV_INT8, lens=[150, 70], q_lens=[10, 7], H=24, Hk=3,
                             D=128, bs=16)
@@ -93,6 +94,25 @@ def test_non_causal_bf16():
     prob, _ = paged_problem(rng, kv_dtype=KV_INT8, lens=[333, 64, 90], q_lens=[12, 6, 16], H=32,
                             Hk=8, D=128, bs=32, causal=0)
     _run_checked(_as_workload(prob, 1, 1))
+
+
+@pytest.mark.parametrize("split_blocks", [-1, 5])
+def test_fp32_output(split_blocks):
+    """out_dtype PA_F32: unrounded rows, unsplit and through the combine."""
+    rng = np.random.default_rng(645)
+    prob, _ = paged_problem(rng, kv_dtype=KV_INT8, lens=[410, 70, 129], q_lens=[11, 3, 16], H=32,
+                            Hk=8, D=128, bs=16)
+    _run_checked(_as_workload(prob, 0, 2), split_blocks=split_blocks)
+
+
+def test_every_row_padding_and_tile_edge():
+    """Units of 4..64 rows (R padded to 16, 32, 48, 64) with lengths at the
+    128-key tile edges (127, 128, 129, 256, 257)."""
+    rng = np.random.default_rng(646)
+    lens = [127, 128, 129, 256, 257, 300, 64, 200]
+    ql = [1, 4, 5, 8, 9, 12, 13, 16]
+    prob, _ = paged_problem(rng, kv_dtype=KV_INT8, lens=lens, q_lens=ql, H=32, Hk=8, D=128, bs=16)
+    _run_checked(_as_workload(prob))
 
 
 def test_c4_workload_small():

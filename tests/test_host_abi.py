@@ -70,9 +70,9 @@ def test_plan_zero_new_tokens_everywhere_is_a_no_op():
 def _count_items(cu, L, G, Hk, bs, rows, T, max_splits):
     """Work items by the documented split rule: a sequence with n KV blocks gets
     s = min(max_splits, ceil(n / T)) splits of ceil(n / s) blocks (empty ones
-    dropped), times its groups of KV heads (4 per item; 2 for the 64-row items
+    dropped), times its groups of KV heads (4 per item; 1 for the 64-row items
     of the tensor-core prefill kernel) times its row groups."""
-    hp = 2 if rows == 64 else 4
+    hp = 1 if rows == 64 else 4
     total, most = 0, 1
     for b in range(len(L)):
         qb = int(cu[b + 1] - cu[b])
