@@ -35,8 +35,9 @@
 //                range), takes each row's maximum over the warp's 32 keys by a
 //                halving shuffle exchange (lane j ends with row j) and over the
 //                group's four warps through shared memory, raises the row's
-//                running maximum only when a logit exceeds it by more than 2^8
-//                (then the row's O^T column and partial sums are rescaled), and
+//                running maximum only when a logit exceeds it by more than a
+//                factor 2^15 (then the row's O^T column and partial sums are
+//                rescaled), and
 //                writes its
 //                key's fp16 P^T row; at the end the group sums its row totals,
 //                normalises, applies the V scale and stores its rows (or an
@@ -45,7 +46,8 @@
 //
 // Numerics follow the decode kernel: logits exact up to the digit split of the
 // folded query (error <= 2^-21 of max|q'| sum|k|), fp32 accumulation, P in
-// fp16 (<= 2^8), the V scale applied once at the end.
+// fp16 (<= 2^15, below the fp16 maximum 65504), the V scale applied once at the
+// end.
 //
 // Sources: INT8 codes kept raw and converted to FP16 for the tensor-core MMA
 // with FP32 accumulation, and tensor cores for the prefill tiles (INT8-KV
@@ -254,10 +256,10 @@ __global__ void __launch_bounds__(kPrepThreads) pa_pf_prep_kernel(const FwdArgs 
   __shared__ float ks[kPfD];
   __shared__ float wmax[kPrepThreads / 32];
   __shared__ int bad_scale;
-  // The prefill kernel is launched as this grid's programmatic dependent but is
-  // released only when every CTA here has finished (no launch_dependents): its
-  // CTAs would otherwise hold every SM's shared memory and registers while
-  // waiting for this grid.
+  // The prefill kernel, this grid's programmatic dependent, may start now: it
+  // builds its work order while this grid runs and waits for the grid before
+  // reading the digit units.
+  asm volatile("griddepcontrol.launch_dependents;");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int u = blockIdx.x;  // ((b * Hk + h) * num_row_groups + rg)
   const int rg = u % a.num_row_groups;
@@ -424,8 +426,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // Inputs may come from the previous kernel in the stream (programmatic launch).
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // This grid may start while the pre-pass (its programmatic primary) runs: the
+  // set-up above and the producer's work order touch only inputs; every role
+  // that reads the pre-pass's units, uses the work counter or writes results
+  // waits for the primary first.
   asm volatile("griddepcontrol.launch_dependents;");
 
   if (warp == 0) {
@@ -526,6 +530,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const int qb = __ldg(a.cu_seqlens_q + fb + 1) - q0;
       return pf_decode_item<BS>(a, fb, w - base, q0, qb, __ldg(a.seqlens_k + fb), d);
     };
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     int uses0 = 0, uses1 = 0;  // descriptors published in slot 0 / 1
     int slot = 0;
     int g = 0;                 // tiles issued (stage s armed (g + 2 - s) / 3 times)
@@ -786,6 +791,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
   } else if (warp >= kSmWarp0 && warp < kSmWarp0 + kSmWarps) {
     // ======================================================== softmax / epilogue
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int grp = (warp - kSmWarp0) >> 2;  // row chunks grp and grp + 2
     const int v = warp & 3;                  // TMEM sub-partition: keys (dims) 32 v .. 32 v + 31
     const int kl = 32 * v + lane;            // this thread's key of a tile, dim of the output
@@ -955,7 +961,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         {
           const float tmax = fmaxf(fmaxf(rp[lane], rp[32 + lane]), fmaxf(rp[64 + lane], rp[96 + lane]));
           const float m_old = r_m[lane];
-          const bool raise = tmax > m_old + 8.f;  // any visible logit when none yet
+          const bool raise = tmax > m_old + 15.f;  // any visible logit when none yet
           const float m_new = raise ? tmax : m_old;
           r_m[lane] = m_new;
           r_mu[lane] = (m_new == -INFINITY) ? 0.f : m_new;
@@ -1087,7 +1093,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         __syncwarp();
         const float vs = reinterpret_cast<const float*>(smem + kVScaleOff + dslot * kPfD * 4)[kl];
-#pragma unroll
+#pragma unroll 1
         for (int jc = 0; jc < 2; ++jc) {
           if (jc == 1 && !n1) continue;
           uint32_t o[16];
