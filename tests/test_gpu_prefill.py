@@ -55,7 +55,7 @@ def _run_checked(w, **over):
 
 @pytest.mark.parametrize("bs", [16, 32])
 def test_ragged_causal_prefill(bs):
-    """Lengths around the 64-key tile and the block edges, q_len 0..16."""
+    """Lengths around the 64- and 128-key marks and the block edges, q_len 0..16."""
     rng = np.random.default_rng(500 + bs)
     lens = [5, 64, 65, 130, 0, 191, 300, 17, 1000, 48]
     ql = [5, 16, 7, 12, 0, 16, 1, 17 - 1, 13, 9]
