@@ -129,13 +129,18 @@ typedef struct {
   int max_query_len;      /* exact max_b (cu[b+1] - cu[b]) */
   int max_seqlen_k;       /* max_b seqlens_k[b] */
   int rows_per_cta;       /* query rows (tokens x group heads) per work item: 4, 8
-                             or 16 (4: at most 4 rows per sequence and KV head) */
+                             or 16 (4: at most 4 rows per sequence and KV head),
+                             or 64: the tensor-core prefill kernel, chosen when a
+                             unit has more than 16 rows over an INT8 cache with
+                             head_size 128 and batch <= 1024 */
   int num_row_groups;     /* ceil(max_query_len * H/Hk / rows_per_cta) */
   int num_splits;         /* most KV splits of any sequence (1 = no split); the
                              workspace holds this many partials per row */
   int blocks_per_split;   /* split target T in KV blocks: a sequence with n blocks
                              is cut into min(num_splits, ceil(n / T)) equal splits */
-  int num_work_items;     /* work items (sequence, KV head, row group, split) */
+  int num_work_items;     /* work items (sequence, KV heads, row group, split): four
+                             KV heads per item on the 4/8/16-row kernel, one on
+                             the prefill kernel */
   size_t workspace_bytes; /* bytes the forward call needs (>= 256) */
   /* ---- supplied by the caller before paged_attn_forward ---- */
   void* workspace;        /* device memory, 256-byte aligned, >= workspace_bytes,
